@@ -1,0 +1,270 @@
+/*
+ * CPU oracle for the mixed-bitwidth (EXL2-style) quantised matrix multiply.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header or table with the CUDA library.
+ *
+ * What it computes (plain definitions, slow on purpose):
+ *
+ *   Format (nightvoyager.top exllamav2 report, "核心价值提炼" and "关键设计决策";
+ *   promptquorum "EXL2量化是什么"): the weight matrix W [K x N] (K input rows in
+ *   act-order, N output columns) is quantised with a bitwidth b_j in
+ *   {2,3,4,5,6,8} per 32-row block j, mixing widths inside one layer, with the
+ *   more important rows holding more bits.  Rows are grouped by 128 and each
+ *   (group, column) pair has one fp16 scale (GPTQ lineage, "group 128").
+ *
+ *   Readings taken where the pages are silent:
+ *   - Packed layout: for column n and block j, the 32 codes of the block form
+ *     a 32*b_j-bit little-endian stream, code r at stream bits [r*b_j, r*b_j+b_j).
+ *     Stream bit t is bit (t mod 32) of word row off_j + t/32, where
+ *     off_j = sum_{i<j} b_i; words are stored row-major [sum b][N].
+ *   - Dequantisation is symmetric around the mid code: w = (q - 2^(b-1)) * s.
+ *   - y[m][n] = sum_k x[m][perm[k]] * w[k][n]  (perm[k] is the column of x that
+ *     multiplies W row k).
+ *
+ * Arithmetic: codes are integers, dequantised weights are exact in double
+ * (an 8-bit integer times an fp16 value), sums are accumulated in double in
+ * natural k order.  fp16 <-> double conversions are written out with integer
+ * bit manipulation so no compiler or library rounding is involved.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define ORC_BLOCK 32
+#define ORC_GROUP 128
+
+enum { ORC_OK = 0, ORC_ERR_SHAPE = -2, ORC_ERR_BITS = -3, ORC_ERR_CODE = -9 };
+
+static int width_allowed(int b) {
+    return b == 2 || b == 3 || b == 4 || b == 5 || b == 6 || b == 8;
+}
+
+/* Sum of block widths = number of packed word rows, or a negative error. */
+int64_t oracle_word_rows(const uint8_t *bits, int K) {
+    if (K <= 0 || K % ORC_BLOCK) return ORC_ERR_SHAPE;
+    int64_t s = 0;
+    for (int j = 0; j < K / ORC_BLOCK; ++j) {
+        if (!width_allowed(bits[j])) return ORC_ERR_BITS;
+        s += bits[j];
+    }
+    return s;
+}
+
+/* Word row where each block starts (off_j), computed here independently. */
+static void block_offsets(const uint8_t *bits, int nb, int64_t *off) {
+    int64_t s = 0;
+    for (int j = 0; j < nb; ++j) { off[j] = s; s += bits[j]; }
+}
+
+/* Code of row k, column n, read bit by bit from the packed stream. */
+static uint32_t read_code(const uint32_t *qw, int64_t N, int64_t off, int b, int r, int64_t n) {
+    uint32_t q = 0;
+    for (int t = 0; t < b; ++t) {
+        int64_t p = (int64_t)r * b + t;                 /* stream bit */
+        uint32_t word = qw[(off + p / 32) * N + n];
+        q |= ((word >> (p % 32)) & 1u) << t;
+    }
+    return q;
+}
+
+/* codes [K][N] (uint8, act-order rows) -> qw [sum b][N].  Returns ORC_ERR_CODE
+ * if a code does not fit its block width. */
+int oracle_pack(const uint8_t *codes, const uint8_t *bits, int K, int N, uint32_t *qw) {
+    int64_t rows = oracle_word_rows(bits, K);
+    if (rows < 0) return (int)rows;
+    if (N <= 0) return ORC_ERR_SHAPE;
+    memset(qw, 0, (size_t)rows * (size_t)N * sizeof(uint32_t));
+    int nb = K / ORC_BLOCK;
+    int64_t off = 0;
+    for (int j = 0; j < nb; ++j) {
+        int b = bits[j];
+        for (int r = 0; r < ORC_BLOCK; ++r) {
+            const uint8_t *row = codes + (int64_t)(j * ORC_BLOCK + r) * N;
+            for (int64_t n = 0; n < N; ++n) {
+                uint32_t q = row[n];
+                if (q >> b) return ORC_ERR_CODE;
+                for (int t = 0; t < b; ++t) {
+                    int64_t p = (int64_t)r * b + t;
+                    if ((q >> t) & 1u) qw[(off + p / 32) * N + n] |= 1u << (p % 32);
+                }
+            }
+        }
+        off += b;
+    }
+    return ORC_OK;
+}
+
+/* qw -> codes [K][N]: the inverse of oracle_pack. */
+int oracle_unpack(const uint32_t *qw, const uint8_t *bits, int K, int N, uint8_t *codes) {
+    int64_t rows = oracle_word_rows(bits, K);
+    if (rows < 0) return (int)rows;
+    int nb = K / ORC_BLOCK;
+    int64_t off = 0;
+    for (int j = 0; j < nb; ++j) {
+        for (int r = 0; r < ORC_BLOCK; ++r)
+            for (int64_t n = 0; n < N; ++n)
+                codes[(int64_t)(j * ORC_BLOCK + r) * N + n] = (uint8_t)read_code(qw, N, off, bits[j], r, n);
+        off += bits[j];
+    }
+    return ORC_OK;
+}
+
+/* IEEE binary16 bit pattern -> exact double. */
+double oracle_half_to_double(uint16_t h) {
+    int sign = h >> 15, e = (h >> 10) & 0x1f, m = h & 0x3ff;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);                    /* zero / subnormal */
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + m), e - 25);
+    return sign ? -v : v;
+}
+
+/* double -> binary16, round to nearest, ties to even, by integer arithmetic on
+ * the double's bit pattern (one rounding step). */
+uint16_t oracle_double_to_half(double v) {
+    uint64_t u;
+    memcpy(&u, &v, sizeof u);
+    uint16_t sign = (uint16_t)((u >> 48) & 0x8000);
+    int e2 = (int)((u >> 52) & 0x7ff);
+    uint64_t frac = u & ((1ull << 52) - 1);
+    if (e2 == 0x7ff) return frac ? (uint16_t)(sign | 0x7e00) : (uint16_t)(sign | 0x7c00);
+    if (e2 == 0 && frac == 0) return sign;
+    int e;                 /* value = mant * 2^(e - 52), mant in [2^52, 2^53) */
+    uint64_t mant;
+    if (e2 == 0) {         /* double subnormal: far below fp16 range */
+        return sign;
+    }
+    e = e2 - 1023;
+    mant = frac | (1ull << 52);
+    if (e > 15) return (uint16_t)(sign | 0x7c00);
+    /* Units of the result's last place: 2^(e-10) for normal fp16, 2^-24 for
+     * subnormal fp16.  shift = number of low mantissa bits dropped. */
+    int shift = (e >= -14) ? 42 : 28 - e;
+    if (shift > 53) return sign;        /* < half of the smallest subnormal */
+    uint64_t q = mant >> shift;
+    uint64_t rem = mant & ((1ull << shift) - 1);
+    uint64_t half = 1ull << (shift - 1);
+    if (rem > half || (rem == half && (q & 1))) ++q;
+    if (e >= -14) {
+        if (q == 2048) { q = 1024; ++e; }
+        if (e > 15) return (uint16_t)(sign | 0x7c00);
+        return (uint16_t)(sign | ((uint16_t)(e + 15) << 10) | (uint16_t)(q & 0x3ff));
+    }
+    return (uint16_t)(sign | (uint16_t)q);   /* q == 1024 encodes the smallest normal */
+}
+
+/* w[k][n] = (q - 2^(b-1)) * s[k/128][n], exact in double. */
+int oracle_dequant_f64(const uint32_t *qw, const uint16_t *scales, const uint8_t *bits,
+                       int K, int N, double *w) {
+    int64_t rows = oracle_word_rows(bits, K);
+    if (rows < 0) return (int)rows;
+    int nb = K / ORC_BLOCK;
+    int64_t off = 0;
+    for (int j = 0; j < nb; ++j) {
+        int b = bits[j];
+        for (int r = 0; r < ORC_BLOCK; ++r) {
+            int k = j * ORC_BLOCK + r;
+            for (int64_t n = 0; n < N; ++n) {
+                int q = (int)read_code(qw, N, off, b, r, n);
+                double s = oracle_half_to_double(scales[(int64_t)(k / ORC_GROUP) * N + n]);
+                w[(int64_t)k * N + n] = (double)(q - (1 << (b - 1))) * s;
+            }
+        }
+        off += b;
+    }
+    return ORC_OK;
+}
+
+/* The fp16 dequantised matrix: each exact weight rounded once (RNE). */
+int oracle_dequant_f16(const uint32_t *qw, const uint16_t *scales, const uint8_t *bits,
+                       int K, int N, uint16_t *w16) {
+    int64_t rows = oracle_word_rows(bits, K);
+    if (rows < 0) return (int)rows;
+    double *w = (double *)malloc((size_t)K * (size_t)N * sizeof(double));
+    if (!w) return -100;
+    oracle_dequant_f64(qw, scales, bits, K, N, w);
+    for (int64_t i = 0; i < (int64_t)K * N; ++i) w16[i] = oracle_double_to_half(w[i]);
+    free(w);
+    return ORC_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * y[m][c] = sum_k x[m][perm[k]] * w[k][col_c], double accumulation in natural
+ * k order.  Columns col_c = cols[c] (or c when cols == NULL).  The column list
+ * is split across threads; each thread handles whole columns.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    const double *x; const int32_t *perm; const uint32_t *qw; const uint16_t *scales;
+    const uint8_t *bits; const int64_t *off; const int64_t *cols;
+    int M, K; int64_t N, ncols, c0, c1; double *y;
+} gemm_job;
+
+static void *gemm_worker(void *arg) {
+    gemm_job *J = (gemm_job *)arg;
+    int nb = J->K / ORC_BLOCK;
+    double *acc = (double *)malloc(sizeof(double) * (size_t)J->M);
+    for (int64_t c = J->c0; c < J->c1; ++c) {
+        int64_t n = J->cols ? J->cols[c] : c;
+        for (int m = 0; m < J->M; ++m) acc[m] = 0.0;
+        for (int j = 0; j < nb; ++j) {
+            int b = J->bits[j];
+            for (int r = 0; r < ORC_BLOCK; ++r) {
+                int k = j * ORC_BLOCK + r;
+                int q = (int)read_code(J->qw, J->N, J->off[j], b, r, n);
+                double s = oracle_half_to_double(J->scales[(int64_t)(k / ORC_GROUP) * J->N + n]);
+                double w = (double)(q - (1 << (b - 1))) * s;
+                int32_t src = J->perm[k];
+                for (int m = 0; m < J->M; ++m) acc[m] += J->x[(int64_t)m * J->K + src] * w;
+            }
+        }
+        for (int m = 0; m < J->M; ++m) J->y[(int64_t)m * J->ncols + c] = acc[m];
+    }
+    free(acc);
+    return NULL;
+}
+
+/* x: double [M][K]; perm: int32 [K] (a permutation of 0..K-1); qw: [sum b][N];
+ * scales: fp16 bits [ceil(K/128)][N]; y: double [M][ncols].
+ * nthreads <= 0 uses every online core.  Returns the thread count used, or a
+ * negative error. */
+int oracle_qgemm_f64(const double *x, const int32_t *perm, const uint32_t *qw,
+                     const uint16_t *scales, const uint8_t *bits, int M, int K, int N,
+                     const int64_t *cols, int64_t ncols, double *y, int nthreads) {
+    int64_t rows = oracle_word_rows(bits, K);
+    if (rows < 0) return (int)rows;
+    if (M <= 0 || N <= 0) return ORC_ERR_SHAPE;
+    for (int k = 0; k < K; ++k)
+        if (perm[k] < 0 || perm[k] >= K) return ORC_ERR_SHAPE;
+    if (!cols) ncols = N;
+    int nb = K / ORC_BLOCK;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)nb);
+    block_offsets(bits, nb, off);
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > ncols) nthreads = (int)ncols;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    gemm_job *jobs = (gemm_job *)malloc(sizeof(gemm_job) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) {
+        gemm_job J = {x, perm, qw, scales, bits, off, cols, M, K, N, ncols,
+                      ncols * t / nthreads, ncols * (t + 1) / nthreads, y};
+        jobs[t] = J;
+        pthread_create(&th[t], NULL, gemm_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+    free(th); free(jobs); free(off);
+    return nthreads;
+}
+
+/* Array forms of the two conversions, for the tests. */
+void oracle_half_to_double_n(const uint16_t *h, double *v, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) v[i] = oracle_half_to_double(h[i]);
+}
+
+void oracle_double_to_half_n(const double *v, uint16_t *h, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) h[i] = oracle_double_to_half(v[i]);
+}
