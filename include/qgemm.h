@@ -1,0 +1,160 @@
+/*
+ * qgemm.h — C ABI of the mixed-bitwidth (EXL2-style) quantised matrix multiply
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  y = x[:, perm] . dequant(Wq):
+ *   - W is K x N (K input rows in act-order, N output columns).  Its rows are cut
+ *     into 32-row blocks; block j is quantised at b_j bits, b_j in {2,3,4,5,6,8},
+ *     widths mixed inside one matrix to hit a target average bits-per-weight,
+ *     more important (act-order-first) rows holding more bits
+ *     (nightvoyager.top exllamav2 report, "核心价值提炼" / "关键设计决策";
+ *     promptquorum "EXL2量化是什么").
+ *   - Each (128-row group, column) pair has one fp16 scale (GPTQ "group 128"
+ *     lineage, ainews.cool ExLlamaV3 article, benchmark table).
+ *   - w[k][n] = (q[k][n] - 2^(b_j - 1)) * s[k/128][n]           (symmetric codes)
+ *   - y[m][n] = sum_k x[m][perm[k]] * w[k][n], fp32 accumulation, fp16 result.
+ * The pages give no bit layout; this library uses (and documents as) the
+ * following one.  For column n and block j the 32 codes form a little-endian
+ * bit stream of 32*b_j bits, code r in stream bits [r*b_j, r*b_j + b_j); stream
+ * bit t is bit (t mod 32) of word row off_j + t/32, off_j = sum_{i<j} b_i.
+ * Words are stored row-major, qw[row][n], so one word row is N contiguous
+ * uint32 values.
+ *
+ * Conventions for every device call:
+ *   - d_* pointers are device memory owned by the caller; h_* pointers are host
+ *     memory.  The library never allocates, frees or synchronises; each call is
+ *     asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - fp16 values are passed as uint16_t bit patterns (IEEE binary16).
+ *   - Shapes: K % 32 == 0, N % 8 == 0, M >= 1, K <= 65536, N <= 2^24.
+ *     Every device pointer must be 16-byte aligned.
+ *   - Schedule: d_bits[K/32] holds b_j, d_offs[K/32 + 1] its prefix sums
+ *     (d_offs[0] = 0, d_offs[K/32] = qw_rows).  qgemm_offsets() computes them on
+ *     the host.  Kernels read the table before touching the weights and refuse
+ *     an inconsistent one (see qgemm_device_error()).
+ *   - Return value: QGEMM_OK, or a negative qgemm_status for an argument error
+ *     found on the host (nothing is launched) or a launch failure
+ *     (QGEMM_ERR_CUDA).  Errors found on the device (an inconsistent schedule,
+ *     perm out of range, a pipeline wait that timed out) make the kernel write
+ *     nothing it should not, record a code in a per-device error word and
+ *     return; read it with qgemm_device_error().  Nothing traps or aborts and
+ *     no C++ exception crosses this boundary.
+ */
+#ifndef QGEMM_H
+#define QGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QGEMM_OK = 0,
+    QGEMM_ERR_NULL = -1,        /* a required pointer is NULL                        */
+    QGEMM_ERR_SHAPE = -2,       /* M, K, N or qw_rows outside the supported range    */
+    QGEMM_ERR_BITS = -3,        /* a block width not in {2,3,4,5,6,8} / bad offsets   */
+    QGEMM_ERR_ALIGN = -4,       /* a device pointer is not 16-byte aligned           */
+    QGEMM_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required        */
+    QGEMM_ERR_DTYPE = -6,       /* x_dtype is not a qgemm_dtype                      */
+    QGEMM_ERR_CUDA = -7,        /* a CUDA runtime call or launch failed              */
+    QGEMM_ERR_UNSUPPORTED = -8  /* valid request this build does not handle          */
+} qgemm_status;
+
+typedef enum { QGEMM_F16 = 0, QGEMM_BF16 = 1 } qgemm_dtype;
+
+/* Device error word codes (qgemm_device_error). */
+#define QGEMM_DEV_OK 0
+#define QGEMM_DEV_BAD_SCHEDULE 1   /* d_bits/d_offs inconsistent or not matching qw_rows */
+#define QGEMM_DEV_BAD_PERM 2       /* a perm entry outside [0, K)                        */
+#define QGEMM_DEV_TIMEOUT 4        /* a pipeline wait gave up after ~1 s                 */
+
+/* ---------------------------------------------------------------- host only */
+
+/* Library version (major*10000 + minor*100 + patch). */
+int qgemm_version(void);
+
+/* Human-readable name of a qgemm_status value (static string). */
+const char* qgemm_status_string(int status);
+
+/* sum_j h_bits[j] over the K/32 blocks = number of packed word rows, or a
+ * negative qgemm_status (QGEMM_ERR_SHAPE for K % 32 != 0, QGEMM_ERR_BITS for a
+ * width outside {2,3,4,5,6,8}). */
+int64_t qgemm_packed_word_rows(const uint8_t* h_bits, int K);
+
+/* Writes h_offs[0..K/32] = prefix sums of h_bits (h_offs[0] = 0).  Returns
+ * QGEMM_OK or a negative status as qgemm_packed_word_rows. */
+int qgemm_offsets(const uint8_t* h_bits, int K, int32_t* h_offs);
+
+/* Checks a host copy of the schedule: widths allowed, offsets equal to their
+ * prefix sums and h_offs[K/32] == qw_rows. */
+int qgemm_validate_schedule(const uint8_t* h_bits, const int32_t* h_offs, int K, int64_t qw_rows);
+
+/* Bytes of workspace qgemm() needs for this shape (0 is possible).  The first
+ * call with a given workspace needs it zero-filled; every completed call leaves
+ * it reusable (its counters return to zero).  Two calls that overlap in time
+ * must not share a workspace. */
+size_t qgemm_workspace_bytes(int M, int K, int N);
+
+/* Number of bytes the packed weights of one K x N matrix occupy:
+ * 4 * N * qw_rows (words) and 2 * N * ceil(K/128) (scales). */
+size_t qgemm_packed_bytes(int64_t qw_rows, int N);
+size_t qgemm_scale_bytes(int K, int N);
+
+/* Reads (and with clear != 0 resets) the device error word of the current CUDA
+ * device.  Synchronises the device. Returns QGEMM_OK or QGEMM_ERR_CUDA. */
+int qgemm_device_error(int* h_code, int clear);
+
+/* Which kernel family qgemm() uses for M rows: 0 = split-K GEMV (CUDA-core
+ * unpack + mma.sync), 1 = tcgen05 tensor-core GEMM with dequantisation into
+ * shared memory. */
+int qgemm_path_for(int M, int K, int N);
+
+/* Launch plan qgemm() would use for this shape on the current device (or on a
+ * 148-SM device when no GPU is visible).  out[0] = kernel family (as
+ * qgemm_path_for), out[1] = grid size, out[2] = shared-memory ring rows (GEMV),
+ * out[3] = activation-stage capacity in blocks (GEMV), out[4] = dynamic shared
+ * memory bytes, out[5] = SM count used.  Host only; returns a qgemm_status. */
+int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out);
+
+/* ----------------------------------------------------------- device calls */
+
+/* Pack codes into the layout above.
+ *   d_codes [K][N] uint8, row k = act-order row, value < 2^b_j (higher bits of a
+ *           wider value are ignored);
+ *   d_qw    [qw_rows][N] uint32 output, fully written.
+ * Source: the EXL2 mixed-width format (nightvoyager.top exllamav2 report,
+ * "核心价值提炼"); the bit layout is this library's reading. */
+int qgemm_pack(const uint8_t* d_codes, const uint8_t* d_bits, const int32_t* d_offs,
+               int K, int N, int64_t qw_rows, uint32_t* d_qw, void* stream);
+
+/* Dequantise to fp16: d_w[k][n] = RNE_fp16((q - 2^(b-1)) * s[k/128][n]),
+ * computed exactly before the one rounding (bit-exact with any correct
+ * implementation).  d_scales [ceil(K/128)][N] fp16, d_w [K][N] fp16 (act-order
+ * rows).  Source: per-group scale of the format (nightvoyager.top exllamav2
+ * report, "关键设计决策", AdaptiveQuantizer paragraph). */
+int qgemm_dequant(const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scales,
+                  const uint8_t* d_bits, const int32_t* d_offs, int K, int N,
+                  uint16_t* d_w, void* stream);
+
+/* y = x[:, perm] . dequant(qw)   (the Q-GEMM the pages credit to exllamav2_ext,
+ * nightvoyager.top report "解法哲学"; bandwidth-bound decode per the navi2ai
+ * ExLlamaV3 page, "核心能力").
+ *   d_x      [M][K] fp16 or bf16 (x_dtype), row-major;
+ *   d_perm   [K] int32, perm[k] = column of x that multiplies W row k;
+ *   d_qw     [qw_rows][N] uint32; d_scales [ceil(K/128)][N] fp16;
+ *   d_y      [M][N] fp16 output (RNE of the fp32 sum);
+ *   d_ws     workspace of at least qgemm_workspace_bytes(M, K, N) bytes
+ *            (may be NULL when that is 0).
+ * M <= 16 runs the split-K GEMV, larger M the tcgen05 GEMM (qgemm_path_for). */
+int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
+          const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scales,
+          const uint8_t* d_bits, const int32_t* d_offs,
+          int M, int K, int N, uint16_t* d_y,
+          void* d_ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGEMM_H */

@@ -1,0 +1,196 @@
+"""Python binding of the qgemm C ABI (include/qgemm.h).
+
+Argument marshalling only: every function checks tensor dtypes, devices and
+contiguity, passes raw pointers and the current CUDA stream to the C library,
+and turns a negative status into ``QGemmError``.  All arithmetic runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and importing this
+package fails if ``libqgemm.so`` has not been built (``build()``).
+
+Names follow the C entry points: ``qgemm_pack``, ``qgemm_dequant``, ``qgemm``,
+``qgemm_workspace_bytes``, ``qgemm_packed_word_rows``, ``qgemm_offsets``,
+``qgemm_validate_schedule``, ``qgemm_device_error``, ``qgemm_path_for``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from ._build import LIB as _LIB_PATH
+from ._build import build  # noqa: F401  (re-exported)
+
+QGEMM_F16 = 0
+QGEMM_BF16 = 1
+DEV_BAD_SCHEDULE = 1
+DEV_BAD_PERM = 2
+DEV_TIMEOUT = 4
+
+
+class QGemmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: run mixed_bitwidth_weight_b200.build() "
+                          "(or __graft_entry__.build()) first")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "qgemm_version": (I, []),
+        "qgemm_status_string": (ctypes.c_char_p, [I]),
+        "qgemm_packed_word_rows": (I64, [P, I]),
+        "qgemm_offsets": (I, [P, I, P]),
+        "qgemm_validate_schedule": (I, [P, P, I, I64]),
+        "qgemm_workspace_bytes": (SZ, [I, I, I]),
+        "qgemm_packed_bytes": (SZ, [I64, I]),
+        "qgemm_scale_bytes": (SZ, [I, I]),
+        "qgemm_device_error": (I, [P, I]),
+        "qgemm_path_for": (I, [I, I, I]),
+        "qgemm_plan_info": (I, [I, I, I, I64, P]),
+        "qgemm_pack": (I, [P, P, P, I, I, I64, P, P]),
+        "qgemm_dequant": (I, [P, I64, P, P, P, I, I, P, P]),
+        "qgemm": (I, [P, I, P, P, I64, P, P, P, I, I, I, P, P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+LIBRARY_PATH = _LIB_PATH
+
+
+def status_string(status: int) -> str:
+    return _lib.qgemm_status_string(int(status)).decode()
+
+
+def _ok(status: int, where: str) -> int:
+    if status < 0:
+        raise QGemmError(int(status), where)
+    return status
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, dtype, name):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_u8(a):
+    return np.ascontiguousarray(np.asarray(a), dtype=np.uint8)
+
+
+# ------------------------------------------------------------- host helpers
+
+def qgemm_version() -> int:
+    return _lib.qgemm_version()
+
+
+def qgemm_packed_word_rows(bits, K: int) -> int:
+    b = _host_u8(bits)
+    return _ok(_lib.qgemm_packed_word_rows(ctypes.c_void_p(b.ctypes.data), K), "qgemm_packed_word_rows")
+
+
+def qgemm_offsets(bits, K: int) -> np.ndarray:
+    b = _host_u8(bits)
+    out = np.empty(K // 32 + 1, dtype=np.int32)
+    _ok(_lib.qgemm_offsets(ctypes.c_void_p(b.ctypes.data), K, ctypes.c_void_p(out.ctypes.data)),
+        "qgemm_offsets")
+    return out
+
+
+def qgemm_validate_schedule(bits, offs, K: int, qw_rows: int) -> int:
+    b = _host_u8(bits)
+    o = np.ascontiguousarray(np.asarray(offs), dtype=np.int32)
+    return _lib.qgemm_validate_schedule(ctypes.c_void_p(b.ctypes.data), ctypes.c_void_p(o.ctypes.data),
+                                        K, int(qw_rows))
+
+
+def qgemm_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(_lib.qgemm_workspace_bytes(M, K, N))
+
+
+def qgemm_path_for(M: int, K: int, N: int) -> int:
+    return int(_lib.qgemm_path_for(M, K, N))
+
+
+def qgemm_plan_info(M: int, K: int, N: int, qw_rows: int) -> dict:
+    out = (ctypes.c_int64 * 6)()
+    _ok(_lib.qgemm_plan_info(M, K, N, int(qw_rows), out), "qgemm_plan_info")
+    return dict(path=out[0], grid=out[1], ring=out[2], span_cap=out[3], smem=out[4], sms=out[5])
+
+
+def qgemm_device_error(clear: bool = True) -> int:
+    code = ctypes.c_int(0)
+    _ok(_lib.qgemm_device_error(ctypes.byref(code), 1 if clear else 0), "qgemm_device_error")
+    return code.value
+
+
+# ------------------------------------------------------------- device calls
+
+def qgemm_pack(codes, bits, offs, qw, stream=None):
+    """codes uint8 [K, N] -> qw int32/uint32 [qw_rows, N] (all CUDA tensors)."""
+    import torch
+    K, N = codes.shape
+    rows = qw.shape[0]
+    _ok(_lib.qgemm_pack(_dev(codes, torch.uint8, "codes"), _dev(bits, torch.uint8, "bits"),
+                        _dev(offs, torch.int32, "offs"), K, N, rows,
+                        _dev(qw, (torch.int32, torch.uint32), "qw"), _stream(stream)), "qgemm_pack")
+    return qw
+
+
+def qgemm_dequant(qw, scales, bits, offs, w, stream=None):
+    """qw [qw_rows, N], scales fp16 [ceil(K/128), N] -> w fp16 [K, N]."""
+    import torch
+    K, N = w.shape
+    _ok(_lib.qgemm_dequant(_dev(qw, (torch.int32, torch.uint32), "qw"), qw.shape[0],
+                           _dev(scales, torch.float16, "scales"), _dev(bits, torch.uint8, "bits"),
+                           _dev(offs, torch.int32, "offs"), K, N, _dev(w, torch.float16, "w"),
+                           _stream(stream)), "qgemm_dequant")
+    return w
+
+
+def qgemm(x, perm, qw, scales, bits, offs, y, ws=None, stream=None):
+    """y [M, N] fp16 = x[:, perm] . dequant(qw); x fp16 or bf16 [M, K]."""
+    import torch
+    M, K = x.shape
+    N = y.shape[1]
+    if x.dtype == torch.float16:
+        xdt = QGEMM_F16
+    elif x.dtype == torch.bfloat16:
+        xdt = QGEMM_BF16
+    else:
+        raise TypeError("x must be float16 or bfloat16")
+    if ws is None:
+        wsp, wsb = ctypes.c_void_p(0), 0
+    else:
+        wsp, wsb = _dev(ws, torch.uint8, "ws"), ws.numel()
+    _ok(_lib.qgemm(_dev(x, None, "x"), xdt, _dev(perm, torch.int32, "perm"),
+                   _dev(qw, (torch.int32, torch.uint32), "qw"), qw.shape[0],
+                   _dev(scales, torch.float16, "scales"), _dev(bits, torch.uint8, "bits"),
+                   _dev(offs, torch.int32, "offs"), M, K, N, _dev(y, torch.float16, "y"),
+                   wsp, wsb, _stream(stream)), "qgemm")
+    return y
+
+
+def workspace(M: int, K: int, N: int, device="cuda"):
+    """A zero-filled workspace tensor of the size qgemm needs for this shape."""
+    import torch
+    return torch.zeros(max(16, qgemm_workspace_bytes(M, K, N)), dtype=torch.uint8, device=device)

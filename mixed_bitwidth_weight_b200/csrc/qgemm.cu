@@ -1,0 +1,318 @@
+// C-ABI entry points of the qgemm library (see include/qgemm.h).
+//
+// This file is the library's only translation unit: it includes the kernels,
+// validates every argument on the host before anything is launched, sizes the
+// launches for the current device and maps CUDA failures to qgemm_status.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace {
+
+using namespace qg;
+
+constexpr int kVersion = 100;  // 0.1.0
+
+struct DeviceInfo {
+    int sms = 0;
+    bool gemv_attr[2] = {false, false};
+};
+
+DeviceInfo g_devs[64];
+std::mutex g_dev_mu;
+
+int current_device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QGEMM_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& d = g_devs[dev];
+    if (d.sms == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return QGEMM_ERR_CUDA;
+        d.sms = sms;
+    }
+    *out = &d;
+    return QGEMM_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int K, int N) {
+    if (K <= 0 || K % kBlockRows != 0 || K > kMaxK) return QGEMM_ERR_SHAPE;
+    if (N <= 0 || N % 8 != 0 || N > (1 << 24)) return QGEMM_ERR_SHAPE;
+    return QGEMM_OK;
+}
+
+int check_rows(int K, int64_t qw_rows) {
+    const int64_t nb = K / kBlockRows;
+    if (qw_rows < 2 * nb || qw_rows > 8 * nb) return QGEMM_ERR_SHAPE;
+    return QGEMM_OK;
+}
+
+int launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QGEMM_OK : QGEMM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ GEMV
+int gemv_mt(int M) { return M <= 8 ? 1 : 2; }
+int gemv_tiles(int N) { return (N + kGemvTileCols - 1) / kGemvTileCols; }
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t gemv_fixed_smem(int nb) {
+    return align_up((size_t)(nb + 1) * 4, 16) + 2 * kGemvSlots * 8 + 128;
+}
+
+// Largest grid the GEMV may use (bounds the workspace).
+int64_t gemv_max_grid(int K, int N, int sms) {
+    const int64_t U = (int64_t)gemv_tiles(N) * (K / kBlockRows);
+    return std::min<int64_t>(U, (int64_t)4 * sms);
+}
+
+size_t gemv_workspace(int M, int K, int N, int sms) {
+    const size_t tickets = align_up((size_t)gemv_tiles(N) * 4, 256);
+    const size_t slot = (size_t)gemv_mt(M) * 8 * kGemvTileCols * 4;
+    return tickets + (size_t)gemv_max_grid(K, N, sms) * 2 * slot;
+}
+
+struct GemvPlan {
+    int grid = 0, ring = 0, span_cap = 0;
+    size_t smem = 0;
+};
+
+int plan_gemv(int M, int K, int N, int64_t qw_rows, int sms, GemvPlan* plan) {
+    const int nb = K / kBlockRows;
+    const int64_t U = (int64_t)gemv_tiles(N) * nb;
+    const int64_t C = (int64_t)gemv_tiles(N) * qw_rows;
+    const int64_t gmax = gemv_max_grid(K, N, sms);
+    for (int64_t G = std::min<int64_t>(U, sms); G <= gmax; G = std::min<int64_t>(gmax, G * 2)) {
+        const int64_t max_units = (C / G + 1) / 2 + 2;
+        const int span = (int)std::min<int64_t>(nb, max_units);
+        const size_t xb = align_up((size_t)span * M * 64, 16);
+        const size_t fixed = gemv_fixed_smem(nb);
+        if (fixed + xb + (size_t)kGemvMinRing * kGemvRowBytes <= (size_t)kGemvSmemBudget) {
+            const int ring = (int)std::min<size_t>(kGemvMaxRing,
+                                                   (kGemvSmemBudget - fixed - xb) / kGemvRowBytes);
+            plan->grid = (int)G;
+            plan->ring = ring;
+            plan->span_cap = span;
+            plan->smem = fixed + xb + (size_t)ring * kGemvRowBytes;
+            return QGEMM_OK;
+        }
+        if (G == gmax) break;
+    }
+    return QGEMM_ERR_UNSUPPORTED;
+}
+
+int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
+             const uint16_t* scales, const uint8_t* bits, const int32_t* offs, int M, int K, int N,
+             uint16_t* y, void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev) {
+    GemvPlan plan;
+    int st = plan_gemv(M, K, N, qw_rows, dev->sms, &plan);
+    if (st != QGEMM_OK) return st;
+    if (ws_bytes < gemv_workspace(M, K, N, dev->sms) || ws == nullptr) return QGEMM_ERR_WORKSPACE;
+    const int mt = gemv_mt(M);
+    if (!dev->gemv_attr[mt - 1]) {
+        cudaError_t e = (mt == 1)
+            ? cudaFuncSetAttribute(gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvSmemBudget)
+            : cudaFuncSetAttribute(gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvSmemBudget);
+        if (e != cudaSuccess) return QGEMM_ERR_CUDA;
+        dev->gemv_attr[mt - 1] = true;
+    }
+    GemvParams p;
+    p.x = x;
+    p.perm = perm;
+    p.qw = qw;
+    p.qw_rows = qw_rows;
+    p.scales = reinterpret_cast<const __half*>(scales);
+    p.bits = bits;
+    p.offs = offs;
+    p.y = reinterpret_cast<__half*>(y);
+    p.tickets = reinterpret_cast<int*>(ws);
+    p.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                       align_up((size_t)gemv_tiles(N) * 4, 256));
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.nb = K / kBlockRows;
+    p.tiles = gemv_tiles(N);
+    p.x_bf16 = (x_dtype == QGEMM_BF16);
+    p.ring_rows = plan.ring;
+    p.span_cap = plan.span_cap;
+    if (mt == 1)
+        gemv_kernel<1><<<plan.grid, kGemvThreads, plan.smem, stream>>>(p);
+    else
+        gemv_kernel<2><<<plan.grid, kGemvThreads, plan.smem, stream>>>(p);
+    return launch_status();
+}
+
+}  // namespace
+
+// =========================================================== C ABI
+extern "C" {
+
+int qgemm_version(void) { return kVersion; }
+
+const char* qgemm_status_string(int status) {
+    switch (status) {
+        case QGEMM_OK: return "ok";
+        case QGEMM_ERR_NULL: return "null pointer";
+        case QGEMM_ERR_SHAPE: return "unsupported shape";
+        case QGEMM_ERR_BITS: return "invalid bit schedule";
+        case QGEMM_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case QGEMM_ERR_WORKSPACE: return "workspace missing or too small";
+        case QGEMM_ERR_DTYPE: return "invalid activation dtype";
+        case QGEMM_ERR_CUDA: return "CUDA error";
+        case QGEMM_ERR_UNSUPPORTED: return "unsupported request";
+        default: return "unknown status";
+    }
+}
+
+int64_t qgemm_packed_word_rows(const uint8_t* h_bits, int K) {
+    if (!h_bits) return QGEMM_ERR_NULL;
+    if (K <= 0 || K % kBlockRows != 0 || K > kMaxK) return QGEMM_ERR_SHAPE;
+    int64_t s = 0;
+    for (int j = 0; j < K / kBlockRows; ++j) {
+        const int b = h_bits[j];
+        if (!(b == 2 || b == 3 || b == 4 || b == 5 || b == 6 || b == 8)) return QGEMM_ERR_BITS;
+        s += b;
+    }
+    return s;
+}
+
+int qgemm_offsets(const uint8_t* h_bits, int K, int32_t* h_offs) {
+    if (!h_offs) return QGEMM_ERR_NULL;
+    const int64_t rows = qgemm_packed_word_rows(h_bits, K);
+    if (rows < 0) return (int)rows;
+    int32_t s = 0;
+    for (int j = 0; j < K / kBlockRows; ++j) {
+        h_offs[j] = s;
+        s += h_bits[j];
+    }
+    h_offs[K / kBlockRows] = s;
+    return QGEMM_OK;
+}
+
+int qgemm_validate_schedule(const uint8_t* h_bits, const int32_t* h_offs, int K, int64_t qw_rows) {
+    if (!h_bits || !h_offs) return QGEMM_ERR_NULL;
+    const int64_t rows = qgemm_packed_word_rows(h_bits, K);
+    if (rows < 0) return (int)rows;
+    if (rows != qw_rows) return QGEMM_ERR_BITS;
+    int64_t s = 0;
+    for (int j = 0; j <= K / kBlockRows; ++j) {
+        if (h_offs[j] != s) return QGEMM_ERR_BITS;
+        if (j < K / kBlockRows) s += h_bits[j];
+    }
+    return QGEMM_OK;
+}
+
+size_t qgemm_packed_bytes(int64_t qw_rows, int N) {
+    return qw_rows > 0 && N > 0 ? (size_t)qw_rows * (size_t)N * 4 : 0;
+}
+
+size_t qgemm_scale_bytes(int K, int N) {
+    return K > 0 && N > 0 ? (size_t)((K + kGroupRows - 1) / kGroupRows) * (size_t)N * 2 : 0;
+}
+
+int qgemm_path_for(int M, int K, int N) {
+    (void)K;
+    (void)N;
+    return M <= 16 ? 0 : 1;
+}
+
+size_t qgemm_workspace_bytes(int M, int K, int N) {
+    if (M <= 0 || check_shape(K, N) != QGEMM_OK) return 0;
+    DeviceInfo* dev = nullptr;
+    const int sms = (current_device_info(&dev) == QGEMM_OK) ? dev->sms : 148;
+    if (qgemm_path_for(M, K, N) == 0) return gemv_workspace(M, K, N, sms);
+    return 0;
+}
+
+int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out) {
+    if (!out) return QGEMM_ERR_NULL;
+    int st = check_shape(K, N);
+    if (st != QGEMM_OK) return st;
+    if (M <= 0) return QGEMM_ERR_SHAPE;
+    if ((st = check_rows(K, qw_rows)) != QGEMM_OK) return st;
+    DeviceInfo* dev = nullptr;
+    const int sms = (current_device_info(&dev) == QGEMM_OK) ? dev->sms : 148;
+    for (int i = 0; i < 6; ++i) out[i] = 0;
+    out[0] = qgemm_path_for(M, K, N);
+    out[5] = sms;
+    if (out[0] == 0) {
+        GemvPlan plan;
+        if ((st = plan_gemv(M, K, N, qw_rows, sms, &plan)) != QGEMM_OK) return st;
+        out[1] = plan.grid;
+        out[2] = plan.ring;
+        out[3] = plan.span_cap;
+        out[4] = (int64_t)plan.smem;
+        return QGEMM_OK;
+    }
+    return QGEMM_ERR_UNSUPPORTED;
+}
+
+int qgemm_device_error(int* h_code, int clear) {
+    if (!h_code) return QGEMM_ERR_NULL;
+    if (cudaMemcpyFromSymbol(h_code, qg::g_dev_error, sizeof(int)) != cudaSuccess) return QGEMM_ERR_CUDA;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(qg::g_dev_error, &zero, sizeof(int)) != cudaSuccess) return QGEMM_ERR_CUDA;
+    }
+    return QGEMM_OK;
+}
+
+int qgemm_pack(const uint8_t* d_codes, const uint8_t* d_bits, const int32_t* d_offs, int K, int N,
+               int64_t qw_rows, uint32_t* d_qw, void* stream) {
+    if (!d_codes || !d_bits || !d_offs || !d_qw) return QGEMM_ERR_NULL;
+    int st = check_shape(K, N);
+    if (st != QGEMM_OK) return st;
+    if ((st = check_rows(K, qw_rows)) != QGEMM_OK) return st;
+    if (!aligned16(d_codes) || !aligned16(d_qw)) return QGEMM_ERR_ALIGN;
+    const dim3 grid((N + 127) / 128, K / kBlockRows);
+    pack_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(d_codes, d_bits, d_offs, K, N,
+                                                                      qw_rows, d_qw);
+    return launch_status();
+}
+
+int qgemm_dequant(const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scales,
+                  const uint8_t* d_bits, const int32_t* d_offs, int K, int N, uint16_t* d_w,
+                  void* stream) {
+    if (!d_qw || !d_scales || !d_bits || !d_offs || !d_w) return QGEMM_ERR_NULL;
+    int st = check_shape(K, N);
+    if (st != QGEMM_OK) return st;
+    if ((st = check_rows(K, qw_rows)) != QGEMM_OK) return st;
+    if (!aligned16(d_qw) || !aligned16(d_scales) || !aligned16(d_w)) return QGEMM_ERR_ALIGN;
+    const dim3 grid((N / 4 + 127) / 128, K / kBlockRows);
+    dequant_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        d_qw, qw_rows, reinterpret_cast<const __half*>(d_scales), d_bits, d_offs, K, N,
+        reinterpret_cast<__half*>(d_w));
+    return launch_status();
+}
+
+int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm, const uint32_t* d_qw,
+          int64_t qw_rows, const uint16_t* d_scales, const uint8_t* d_bits,
+          const int32_t* d_offs, int M, int K, int N, uint16_t* d_y, void* d_ws,
+          size_t ws_bytes, void* stream) {
+    if (!d_x || !d_perm || !d_qw || !d_scales || !d_bits || !d_offs || !d_y) return QGEMM_ERR_NULL;
+    if (x_dtype != QGEMM_F16 && x_dtype != QGEMM_BF16) return QGEMM_ERR_DTYPE;
+    int st = check_shape(K, N);
+    if (st != QGEMM_OK) return st;
+    if (M <= 0 || M > (1 << 20)) return QGEMM_ERR_SHAPE;
+    if ((st = check_rows(K, qw_rows)) != QGEMM_OK) return st;
+    if (!aligned16(d_x) || !aligned16(d_perm) || !aligned16(d_qw) || !aligned16(d_scales) ||
+        !aligned16(d_y) || (d_ws && !aligned16(d_ws)))
+        return QGEMM_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    if ((st = current_device_info(&dev)) != QGEMM_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (qgemm_path_for(M, K, N) == 0)
+        return run_gemv(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y,
+                        d_ws, ws_bytes, s, dev);
+    return QGEMM_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+"""The C ABI without a GPU: the library loads, exports every entry point its
+header declares, and its host-side helpers and argument checks behave."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import mixed_bitwidth_weight_b200 as q
+import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgemm.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\**\s+\**\s*(qgemm[a-z_0-9]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = header_functions()
+    for required in ("qgemm", "qgemm_pack", "qgemm_dequant", "qgemm_workspace_bytes",
+                     "qgemm_packed_word_rows", "qgemm_offsets", "qgemm_device_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", q.LIBRARY_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(\S+)$", out, flags=re.M))
+    missing = [n for n in header_functions() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    lib = ctypes.CDLL(q.LIBRARY_PATH)
+    for n in header_functions():
+        assert getattr(lib, n) is not None
+
+
+def test_library_has_no_oracle_dependency():
+    out = subprocess.run(["nm", "-D", q.LIBRARY_PATH], capture_output=True, text=True).stdout
+    assert "oracle" not in out
+    ldd = subprocess.run(["ldd", q.LIBRARY_PATH], capture_output=True, text=True).stdout
+    assert "liboracle" not in ldd and "libtorch" not in ldd
+
+
+def test_version_and_status_strings():
+    assert q.qgemm_version() >= 100
+    for st in range(-8, 1):
+        assert q.status_string(st) and q.status_string(st) != "unknown status"
+    assert q.status_string(-99) == "unknown status"
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_word_rows_and_offsets_match_schedule(name):
+    w = W.WORKLOADS[name]
+    shapes = [(K, N) for _, K, N in w.matrices] if w.matrices else [(w.K, w.N)]
+    for K, N in shapes:
+        bits = W.schedule_for(w, K)
+        assert q.qgemm_packed_word_rows(bits, K) == int(bits.astype(np.int64).sum())
+        offs = q.qgemm_offsets(bits, K)
+        assert np.array_equal(offs, W.offsets(bits))
+        assert q.qgemm_validate_schedule(bits, offs, K, int(offs[-1])) == 0
+
+
+def test_schedule_validation_errors():
+    bits = np.array([4, 2, 8, 3], np.uint8)
+    offs = q.qgemm_offsets(bits, 128)
+    assert q.qgemm_validate_schedule(bits, offs, 128, 16) == -3       # qw_rows mismatch
+    bad = offs.copy()
+    bad[2] += 1
+    assert q.qgemm_validate_schedule(bits, bad, 128, 17) == -3
+    with pytest.raises(q.QGemmError):
+        q.qgemm_packed_word_rows(np.array([7], np.uint8), 32)
+    with pytest.raises(q.QGemmError):
+        q.qgemm_packed_word_rows(np.array([4], np.uint8), 33)
+
+
+def test_workspace_and_sizes():
+    assert q.qgemm_workspace_bytes(1, 8192, 28672) > 0
+    assert q.qgemm_workspace_bytes(0, 8192, 28672) == 0
+    assert q.qgemm_workspace_bytes(1, 33, 64) == 0
+    lib = q._lib
+    assert lib.qgemm_packed_bytes(621, 28672) == 4 * 621 * 28672
+    assert lib.qgemm_scale_bytes(8192, 28672) == 2 * 64 * 28672
+    assert lib.qgemm_scale_bytes(160, 8) == 2 * 2 * 8
+    assert q.qgemm_path_for(1, 8192, 8192) == 0
+    assert q.qgemm_path_for(16, 8192, 8192) == 0
+    assert q.qgemm_path_for(2048, 8192, 8192) == 1
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_host_argument_errors_return_status_without_launching():
+    lib = q._lib
+    A = 0x7f0000000000  # never dereferenced: every case fails before any CUDA call
+    good = dict(x=_fake(A), dt=0, perm=_fake(A), qw=_fake(A), rows=16, s=_fake(A), b=_fake(A),
+                o=_fake(A), M=1, K=128, N=64, y=_fake(A), ws=_fake(A), wsb=1 << 20, st=_fake(0))
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return lib.qgemm(a["x"], a["dt"], a["perm"], a["qw"], a["rows"], a["s"], a["b"], a["o"],
+                         a["M"], a["K"], a["N"], a["y"], a["ws"], a["wsb"], a["st"])
+
+    assert call(x=_fake(0)) == -1
+    assert call(y=_fake(0)) == -1
+    assert call(dt=7) == -6
+    assert call(K=100) == -2
+    assert call(N=60) == -2
+    assert call(M=0) == -2
+    assert call(rows=7) == -2          # fewer than 2 rows per block
+    assert call(rows=33) == -2         # more than 8 rows per block
+    assert call(x=_fake(A + 8)) == -4
+    assert call(qw=_fake(A + 4)) == -4
+    assert lib.qgemm_pack(_fake(0), _fake(A), _fake(A), 128, 64, 16, _fake(A), _fake(0)) == -1
+    assert lib.qgemm_pack(_fake(A), _fake(A), _fake(A), 128, 64, 16, _fake(A + 2), _fake(0)) == -4
+    assert lib.qgemm_dequant(_fake(A), 16, _fake(A), _fake(A), _fake(A), 100, 64, _fake(A), _fake(0)) == -2

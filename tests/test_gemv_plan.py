@@ -1,0 +1,89 @@
+"""Host-side checks of the decode GEMV launch plan, without a GPU.
+
+The kernel splits the (256-column tile, 32-row block) units into contiguous,
+equal-cost ranges, one per CTA (see csrc/gemv.cuh).  This file replays that
+split in Python for the workload shapes and checks what keeps the kernel in
+bounds: every unit is owned by exactly one CTA, the CTA that owns a unit is the
+one the reducer expects (cta_of), a CTA's blocks fit the activation stage the
+plan sized, a unit fits the shared-memory ring, and partial-sum slots stay
+inside the workspace.
+"""
+import bisect
+
+import numpy as np
+import pytest
+
+import mixed_bitwidth_weight_b200 as q
+import workloads as W
+from tests import problems as P
+
+TILE = 256
+
+
+def replay(offs, tiles, G):
+    nb = len(offs) - 1
+    Wr = int(offs[-1])
+    C = tiles * Wr
+
+    def unit_start(i):
+        if i >= G:
+            return tiles * nb
+        pos = (i * C + G - 1) // G
+        t = pos // Wr
+        rem = pos - t * Wr
+        j = bisect.bisect_left(list(offs), rem)
+        return t * nb + j
+
+    def cta_of(u):
+        t, j = divmod(u, nb)
+        return ((t * Wr + int(offs[j])) * G) // C
+
+    return [unit_start(i) for i in range(G + 1)], cta_of
+
+
+def shapes():
+    out = []
+    for name, w in W.WORKLOADS.items():
+        mats = [(K, N) for _, K, N in w.matrices] if w.matrices else [(w.K, w.N)]
+        for K, N in mats:
+            bits = W.schedule_for(w, K)
+            out.append((name, K, N, bits))
+    for K, N in [(32, 8), (160, 264), (1024, 1048), (2048, 4104), (8192, 256), (65536, 8)]:
+        out.append(("small", K, N, P.schedule("shuffled", K // 32, seed=K)))
+        out.append(("small_u2", K, N, W.uniform_schedule(K // 32, 2)))
+        out.append(("small_u8", K, N, W.uniform_schedule(K // 32, 8)))
+    return out
+
+
+@pytest.mark.parametrize("M", [1, 4, 8, 9, 16])
+@pytest.mark.parametrize("case", shapes(), ids=lambda c: f"{c[0]}-{c[1]}x{c[2]}")
+def test_gemv_plan_keeps_kernel_in_bounds(case, M):
+    name, K, N, bits = case
+    offs = W.offsets(bits)
+    nb = K // 32
+    rows = int(offs[-1])
+    tiles = (N + TILE - 1) // TILE
+    plan = q.qgemm_plan_info(M, K, N, rows)
+    assert plan["path"] == 0
+    G = plan["grid"]
+    assert 1 <= G <= 4 * plan["sms"]
+    assert plan["smem"] <= 227 * 1024
+    assert plan["ring"] >= 24
+    starts, cta_of = replay(offs, tiles, G)
+    assert starts[0] == 0 and starts[-1] == tiles * nb
+    assert all(a <= b for a, b in zip(starts, starts[1:]))
+    mt = 1 if M <= 8 else 2
+    ws = q.qgemm_workspace_bytes(M, K, N)
+    slot_bytes = mt * 8 * TILE * 4
+    assert ws >= ((tiles * 4 + 255) // 256 * 256) + G * 2 * slot_bytes
+    rng = np.random.default_rng(K + N + M)
+    for i in range(G):
+        u0, u1 = starts[i], starts[i + 1]
+        n = u1 - u0
+        if n <= 0:
+            continue
+        assert min(nb, n) <= plan["span_cap"], (i, n)
+        for u in {u0, u1 - 1, *rng.integers(u0, u1, size=min(4, n)).tolist()}:
+            assert cta_of(u) == i
+    # a unit (b word rows + one scale row) always fits the ring
+    assert int(bits.max()) + 1 <= plan["ring"]

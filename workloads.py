@@ -151,6 +151,16 @@ def bit_schedule(nb: int, allowed, target_sum: int, seed: int = 0, layer: int = 
     return np.asarray(b, dtype=np.uint8)
 
 
+def random_schedule(nb: int, allowed=ALLOWED_BITS, seed: int = 0, layer: int = 0,
+                    matrix: int = 0) -> np.ndarray:
+    """Unsorted widths drawn uniformly from ``allowed`` (test schedules that a
+    kernel must not assume to be monotone)."""
+    key = stream_key(seed, STREAM_SCHEDULE, layer, matrix ^ 0x80)
+    r = _srl(raw(key, torch.arange(nb)), 11).numpy()
+    A = np.asarray(sorted(allowed), dtype=np.uint8)
+    return A[r % len(A)]
+
+
 def uniform_schedule(nb: int, bits: int) -> np.ndarray:
     return np.full(nb, bits, dtype=np.uint8)
 
