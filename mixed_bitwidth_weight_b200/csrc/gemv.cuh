@@ -421,11 +421,19 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
                 }
         __threadfence();
         named_bar_sync(1, kGemvConsumers);
+        // A CTA between first and last whose range is empty (one unit can cost
+        // more than a CTA's share) contributes nothing and is skipped.
+        auto contributes = [&](int cc) {
+            return unit_start(cc, G, C, W, nb, p.tiles, s_offs) <
+                   unit_start(cc + 1, G, C, W, nb, p.tiles, s_offs);
+        };
         if (ctid == 0) {
             int is_last = 0;
             if (!s_misc[2]) {
+                int n = 0;
+                for (int cc = first; cc <= last; ++cc) n += contributes(cc) ? 1 : 0;
                 const int old = atomicAdd(&p.tickets[tt], 1);
-                is_last = (old == last - first);
+                is_last = (old == n - 1);
             }
             s_misc[1] = is_last;
         }
@@ -438,6 +446,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
                 if (cl >= ncol) continue;
                 float s = 0.f;
                 for (int cc = first; cc <= last; ++cc) {
+                    if (cc != first && cc != last && !contributes(cc)) continue;
                     const int wc = (cc == first && first_before) ? 1 : 0;
                     s += __ldcg(p.slots + ((size_t)cc * 2 + wc) * (MP * kGemvTileCols) +
                                 tok * kGemvTileCols + cl);

@@ -85,5 +85,11 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
         assert min(nb, n) <= plan["span_cap"], (i, n)
         for u in {u0, u1 - 1, *rng.integers(u0, u1, size=min(4, n)).tolist()}:
             assert cta_of(u) == i
+    # the reducer of a tile adds exactly the CTAs that own one of its units
+    for t in range(tiles):
+        owners = {cta_of(u) for u in range(t * nb, (t + 1) * nb)}
+        first, last = cta_of(t * nb), cta_of(t * nb + nb - 1)
+        expect = {c for c in range(first, last + 1) if starts[c] < starts[c + 1]}
+        assert owners == expect, t
     # a unit (b word rows + one scale row) always fits the ring
     assert int(bits.max()) + 1 <= plan["ring"]
