@@ -61,22 +61,35 @@ int launch_status() {
 // ------------------------------------------------------------------ GEMV
 int gemv_mt(int M) { return M <= 8 ? 1 : 2; }
 int gemv_tiles(int N) { return (N + kGemvTileCols - 1) / kGemvTileCols; }
+int gemv_groups(int K) { return (K / kBlockRows + kGemvGroupBlocks - 1) / kGemvGroupBlocks; }
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 size_t gemv_fixed_smem(int nb) {
-    return align_up((size_t)(nb + 1) * 4, 16) + 2 * kGemvSlots * 8 + 128;
+    return align_up((size_t)(nb + 1) * 4, 16) + 2 * kGemvSlots * 8 + 16 + 128;
 }
 
 // Largest grid the GEMV may use (bounds the workspace).
 int64_t gemv_max_grid(int K, int N, int sms) {
-    const int64_t U = (int64_t)gemv_tiles(N) * (K / kBlockRows);
+    const int64_t U = (int64_t)gemv_tiles(N) * gemv_groups(K);
     return std::min<int64_t>(U, (int64_t)4 * sms);
 }
 
-size_t gemv_workspace(int M, int K, int N, int sms) {
-    const size_t tickets = align_up((size_t)gemv_tiles(N) * 4, 256);
-    const size_t slot = (size_t)gemv_mt(M) * 8 * kGemvTileCols * 4;
-    return tickets + (size_t)gemv_max_grid(K, N, sms) * 2 * slot;
+// Workspace: [tickets][partial slots][activations][corrections][row shifts].
+struct GemvWs {
+    size_t tickets, slots, xdec, xcorr, xshift, total;
+};
+
+GemvWs gemv_ws_layout(int M, int K, int N, int sms) {
+    const int mp = gemv_mt(M) * 8;
+    const int nb = K / kBlockRows;
+    GemvWs w;
+    w.tickets = 0;
+    w.slots = align_up((size_t)gemv_tiles(N) * 4, 256);
+    w.xdec = w.slots + align_up((size_t)gemv_max_grid(K, N, sms) * 2 * mp * kGemvTileCols * 4, 256);
+    w.xcorr = w.xdec + align_up((size_t)nb * M * 64, 256);
+    w.xshift = w.xcorr + align_up((size_t)gemv_groups(K) * mp * 4, 256);
+    w.total = w.xshift + 256;
+    return w;
 }
 
 struct GemvPlan {
@@ -86,24 +99,33 @@ struct GemvPlan {
 
 int plan_gemv(int M, int K, int N, int64_t qw_rows, int sms, GemvPlan* plan) {
     const int nb = K / kBlockRows;
-    const int64_t U = (int64_t)gemv_tiles(N) * nb;
-    const int64_t C = (int64_t)gemv_tiles(N) * qw_rows;
+    const int mt = gemv_mt(M);
+    const int64_t U = (int64_t)gemv_tiles(N) * gemv_groups(K);
+    const int64_t C = (int64_t)gemv_tiles(N) * (qw_rows + gemv_groups(K));
     const int64_t gmax = gemv_max_grid(K, N, sms);
-    for (int64_t G = std::min<int64_t>(U, sms); G <= gmax; G = std::min<int64_t>(gmax, G * 2)) {
-        const int64_t max_units = (C / G + 1) / 2 + 2;
-        const int span = (int)std::min<int64_t>(nb, max_units);
-        const size_t xb = align_up((size_t)span * M * 64, 16);
-        const size_t fixed = gemv_fixed_smem(nb);
-        if (fixed + xb + (size_t)kGemvMinRing * kGemvRowBytes <= (size_t)kGemvSmemBudget) {
-            const int ring = (int)std::min<size_t>(kGemvMaxRing,
-                                                   (kGemvSmemBudget - fixed - xb) / kGemvRowBytes);
+    // two CTAs per SM when the activation stage is small (M <= 8), else one
+    const int per_sm = (mt == 1) ? 2 : 1;
+    const size_t budget = (per_sm == 2) ? (size_t)(233472 - 2 * 1024) / 2 : (size_t)227 * 1024;
+    // Every CTA's cost share must hold a whole unit (<= 32 word rows + 1 scale
+    // row), so that no CTA's range is empty: the reduction relies on it.
+    const int64_t gcap = std::max<int64_t>(1, C / (8 * kGemvGroupBlocks + 2));
+    for (int64_t G = std::min<int64_t>(std::min<int64_t>(U, gcap), (int64_t)per_sm * sms); G <= gmax;
+         G = std::min<int64_t>(std::min<int64_t>(gmax, gcap), G * 2)) {
+        // blocks a CTA can touch: each costs >= 2 rows, plus one trailing group
+        const int64_t max_blocks = (C / G + 1) / 2 + kGemvGroupBlocks + 1;  // (scale rows only add cost)
+        const int span = (int)std::min<int64_t>(nb, max_blocks);
+        const size_t xb = (size_t)span * M * 64 +
+                          (size_t)((span + kGemvGroupBlocks - 1) / kGemvGroupBlocks + 1) * mt * 8 * 4;
+        const size_t fixed = align_up(gemv_fixed_smem(nb) + xb, 16);
+        if (fixed + (size_t)kGemvMinRing * kGemvRowBytes <= budget) {
+            const int ring = (int)std::min<size_t>(kGemvMaxRing, (budget - fixed) / kGemvRowBytes);
             plan->grid = (int)G;
             plan->ring = ring;
             plan->span_cap = span;
-            plan->smem = fixed + xb + (size_t)ring * kGemvRowBytes;
+            plan->smem = fixed + (size_t)ring * kGemvRowBytes;
             return QGEMM_OK;
         }
-        if (G == gmax) break;
+        if (G >= std::min<int64_t>(gmax, gcap)) break;
     }
     return QGEMM_ERR_UNSUPPORTED;
 }
@@ -114,39 +136,74 @@ int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     GemvPlan plan;
     int st = plan_gemv(M, K, N, qw_rows, dev->sms, &plan);
     if (st != QGEMM_OK) return st;
-    if (ws_bytes < gemv_workspace(M, K, N, dev->sms) || ws == nullptr) return QGEMM_ERR_WORKSPACE;
+    const GemvWs L = gemv_ws_layout(M, K, N, dev->sms);
+    if (ws_bytes < L.total || ws == nullptr) return QGEMM_ERR_WORKSPACE;
     const int mt = gemv_mt(M);
     if (!dev->gemv_attr[mt - 1]) {
         cudaError_t e = (mt == 1)
-            ? cudaFuncSetAttribute(gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvSmemBudget)
-            : cudaFuncSetAttribute(gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvSmemBudget);
+            ? cudaFuncSetAttribute(gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)
+            : cudaFuncSetAttribute(gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return QGEMM_ERR_CUDA;
         dev->gemv_attr[mt - 1] = true;
     }
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    const int nb = K / kBlockRows;
+
+    XprepParams xp;
+    xp.x = x;
+    xp.perm = perm;
+    xp.bits = bits;
+    xp.offs = offs;
+    xp.xdec = reinterpret_cast<__half*>(w8 + L.xdec);
+    xp.xcorr = reinterpret_cast<float*>(w8 + L.xcorr);
+    xp.xshift = reinterpret_cast<int*>(w8 + L.xshift);
+    xp.M = M;
+    xp.K = K;
+    xp.nb = nb;
+    xp.mp = mt * 8;
+    xp.x_bf16 = (x_dtype == QGEMM_BF16);
+    xprep_kernel<<<(nb + 7) / 8, 256, 0, stream>>>(xp);
+    if ((st = launch_status()) != QGEMM_OK) return st;
+
     GemvParams p;
-    p.x = x;
-    p.perm = perm;
+    p.xdec = xp.xdec;
+    p.xcorr = xp.xcorr;
+    p.xshift = xp.xshift;
     p.qw = qw;
     p.qw_rows = qw_rows;
     p.scales = reinterpret_cast<const __half*>(scales);
     p.bits = bits;
     p.offs = offs;
     p.y = reinterpret_cast<__half*>(y);
-    p.tickets = reinterpret_cast<int*>(ws);
-    p.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                       align_up((size_t)gemv_tiles(N) * 4, 256));
+    p.tickets = reinterpret_cast<int*>(w8 + L.tickets);
+    p.slots = reinterpret_cast<float*>(w8 + L.slots);
     p.M = M;
     p.K = K;
     p.N = N;
-    p.nb = K / kBlockRows;
+    p.nb = nb;
+    p.ng = gemv_groups(K);
     p.tiles = gemv_tiles(N);
-    p.x_bf16 = (x_dtype == QGEMM_BF16);
     p.ring_rows = plan.ring;
     p.span_cap = plan.span_cap;
-    if (mt == 1)
-        gemv_kernel<1><<<plan.grid, kGemvThreads, plan.smem, stream>>>(p);
-    else
-        gemv_kernel<2><<<plan.grid, kGemvThreads, plan.smem, stream>>>(p);
+
+    // launched as a programmatic dependent of xprep: starts streaming weights
+    // while xprep runs and waits for it (griddepcontrol.wait) before reading x
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.grid);
+    cfg.blockDim = dim3(kGemvThreads);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = (mt == 1) ? cudaLaunchKernelEx(&cfg, gemv_kernel<1>, p)
+                                    : cudaLaunchKernelEx(&cfg, gemv_kernel<2>, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return QGEMM_ERR_CUDA;
+    }
     return launch_status();
 }
 
@@ -228,7 +285,7 @@ size_t qgemm_workspace_bytes(int M, int K, int N) {
     if (M <= 0 || check_shape(K, N) != QGEMM_OK) return 0;
     DeviceInfo* dev = nullptr;
     const int sms = (current_device_info(&dev) == QGEMM_OK) ? dev->sms : 148;
-    if (qgemm_path_for(M, K, N) == 0) return gemv_workspace(M, K, N, sms);
+    if (qgemm_path_for(M, K, N) == 0) return gemv_ws_layout(M, K, N, sms).total;
     return 0;
 }
 

@@ -1,6 +1,6 @@
 """Host-side checks of the decode GEMV launch plan, without a GPU.
 
-The kernel splits the (256-column tile, 32-row block) units into contiguous,
+The kernel splits the (256-column tile, 128-row group) units into contiguous,
 equal-cost ranges, one per CTA (see csrc/gemv.cuh).  This file replays that
 split in Python for the workload shapes and checks what keeps the kernel in
 bounds: every unit is owned by exactly one CTA, the CTA that owns a unit is the
@@ -21,24 +21,27 @@ TILE = 256
 
 
 def replay(offs, tiles, G):
+    """The kernel's split: units are (tile, 128-row group), numbered t*ng + g; a
+    unit costs its word rows plus one scale row."""
     nb = len(offs) - 1
-    Wr = int(offs[-1])
-    C = tiles * Wr
+    ng = (nb + 3) // 4
+    Wt = int(offs[-1]) + ng
+    C = tiles * Wt
+    goffs = [int(offs[min(4 * g, nb)]) + g for g in range(ng + 1)]
 
     def unit_start(i):
         if i >= G:
-            return tiles * nb
+            return tiles * ng
         pos = (i * C + G - 1) // G
-        t = pos // Wr
-        rem = pos - t * Wr
-        j = bisect.bisect_left(list(offs), rem)
-        return t * nb + j
+        t = pos // Wt
+        rem = pos - t * Wt
+        return t * ng + bisect.bisect_left(goffs, rem)
 
     def cta_of(u):
-        t, j = divmod(u, nb)
-        return ((t * Wr + int(offs[j])) * G) // C
+        t, g = divmod(u, ng)
+        return ((t * Wt + goffs[g]) * G) // C
 
-    return [unit_start(i) for i in range(G + 1)], cta_of
+    return [unit_start(i) for i in range(G + 1)], cta_of, ng
 
 
 def shapes():
@@ -69,27 +72,29 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     assert 1 <= G <= 4 * plan["sms"]
     assert plan["smem"] <= 227 * 1024
     assert plan["ring"] >= 24
-    starts, cta_of = replay(offs, tiles, G)
-    assert starts[0] == 0 and starts[-1] == tiles * nb
+    starts, cta_of, ng = replay(offs, tiles, G)
+    assert starts[0] == 0 and starts[-1] == tiles * ng
     assert all(a <= b for a, b in zip(starts, starts[1:]))
     mt = 1 if M <= 8 else 2
     ws = q.qgemm_workspace_bytes(M, K, N)
     slot_bytes = mt * 8 * TILE * 4
-    assert ws >= ((tiles * 4 + 255) // 256 * 256) + G * 2 * slot_bytes
+    act_bytes = nb * M * 64 + ((nb + 3) // 4) * mt * 8 * 4 + 64
+    assert ws >= ((tiles * 4 + 255) // 256 * 256) + G * 2 * slot_bytes + act_bytes
     rng = np.random.default_rng(K + N + M)
     for i in range(G):
         u0, u1 = starts[i], starts[i + 1]
         n = u1 - u0
-        if n <= 0:
-            continue
-        assert min(nb, n) <= plan["span_cap"], (i, n)
+        assert n > 0, f"CTA {i} owns no unit (the reduction needs every range non-empty)"
+        blocks = sum(min(4, nb - 4 * (u % ng)) for u in range(u0, u1))
+        assert min(nb, blocks) <= plan["span_cap"], (i, blocks)
         for u in {u0, u1 - 1, *rng.integers(u0, u1, size=min(4, n)).tolist()}:
             assert cta_of(u) == i
     # the reducer of a tile adds exactly the CTAs that own one of its units
     for t in range(tiles):
-        owners = {cta_of(u) for u in range(t * nb, (t + 1) * nb)}
-        first, last = cta_of(t * nb), cta_of(t * nb + nb - 1)
+        owners = {cta_of(u) for u in range(t * ng, (t + 1) * ng)}
+        first, last = cta_of(t * ng), cta_of(t * ng + ng - 1)
         expect = {c for c in range(first, last + 1) if starts[c] < starts[c + 1]}
         assert owners == expect, t
-    # a unit (b word rows + one scale row) always fits the ring
-    assert int(bits.max()) + 1 <= plan["ring"]
+    # a unit (a group's word rows + one scale row) always fits the ring
+    need = max(int(offs[min(4 * g + 4, nb)] - offs[4 * g]) + 1 for g in range(ng))
+    assert need <= plan["ring"]
