@@ -65,7 +65,8 @@ int gemv_groups(int K) { return (K / kBlockRows + kGemvGroupBlocks - 1) / kGemvG
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 size_t gemv_fixed_smem(int nb) {
-    return align_up((size_t)(nb + 1) * 4, 16) + 2 * kGemvSlots * 8 + 16 + 128;
+    size_t o = align_up((size_t)(nb + 1) * 4, 16) + 2 * kGemvSlots * 8 + 2 * kGemvAStages * 8 + 2 * 2 * 8 + 8 + 128;
+    return align_up(o, 128);
 }
 
 // Largest grid the GEMV may use (bounds the workspace).
@@ -74,7 +75,7 @@ int64_t gemv_max_grid(int K, int N, int sms) {
     return std::min<int64_t>(U, (int64_t)4 * sms);
 }
 
-// Workspace: [tickets][partial slots][activations][corrections][row shifts].
+// Workspace: [tickets][partial slots][activation records][corrections][row shifts].
 struct GemvWs {
     size_t tickets, slots, xdec, xcorr, xshift, total;
 };
@@ -86,8 +87,8 @@ GemvWs gemv_ws_layout(int M, int K, int N, int sms) {
     w.tickets = 0;
     w.slots = align_up((size_t)gemv_tiles(N) * 4, 256);
     w.xdec = w.slots + align_up((size_t)gemv_max_grid(K, N, sms) * 2 * mp * kGemvTileCols * 4, 256);
-    w.xcorr = w.xdec + align_up((size_t)nb * M * 64, 256);
-    w.xshift = w.xcorr + align_up((size_t)gemv_groups(K) * mp * 4, 256);
+    w.xcorr = w.xdec + align_up((size_t)(nb + 8) * 64 * mp, 256);
+    w.xshift = w.xcorr + align_up((size_t)(gemv_groups(K) + 2) * mp * 4, 256);
     w.total = w.xshift + 256;
     return w;
 }
@@ -97,37 +98,24 @@ struct GemvPlan {
     size_t smem = 0;
 };
 
+// One CTA per SM (each holds all 512 TMEM columns).  Every CTA's cost share
+// must hold a whole unit (<= 32 word rows + 1 scale row) so that no CTA's
+// range is empty: the reduction relies on it.
 int plan_gemv(int M, int K, int N, int64_t qw_rows, int sms, GemvPlan* plan) {
     const int nb = K / kBlockRows;
-    const int mt = gemv_mt(M);
     const int64_t U = (int64_t)gemv_tiles(N) * gemv_groups(K);
     const int64_t C = (int64_t)gemv_tiles(N) * (qw_rows + gemv_groups(K));
-    const int64_t gmax = gemv_max_grid(K, N, sms);
-    // two CTAs per SM when the activation stage is small (M <= 8), else one
-    const int per_sm = (mt == 1) ? 2 : 1;
-    const size_t budget = (per_sm == 2) ? (size_t)(233472 - 2 * 1024) / 2 : (size_t)227 * 1024;
-    // Every CTA's cost share must hold a whole unit (<= 32 word rows + 1 scale
-    // row), so that no CTA's range is empty: the reduction relies on it.
     const int64_t gcap = std::max<int64_t>(1, C / (8 * kGemvGroupBlocks + 2));
-    for (int64_t G = std::min<int64_t>(std::min<int64_t>(U, gcap), (int64_t)per_sm * sms); G <= gmax;
-         G = std::min<int64_t>(std::min<int64_t>(gmax, gcap), G * 2)) {
-        // blocks a CTA can touch: each costs >= 2 rows, plus one trailing group
-        const int64_t max_blocks = (C / G + 1) / 2 + kGemvGroupBlocks + 1;  // (scale rows only add cost)
-        const int span = (int)std::min<int64_t>(nb, max_blocks);
-        const size_t xb = (size_t)span * M * 64 +
-                          (size_t)((span + kGemvGroupBlocks - 1) / kGemvGroupBlocks + 1) * mt * 8 * 4;
-        const size_t fixed = align_up(gemv_fixed_smem(nb) + xb, 16);
-        if (fixed + (size_t)kGemvMinRing * kGemvRowBytes <= budget) {
-            const int ring = (int)std::min<size_t>(kGemvMaxRing, (budget - fixed) / kGemvRowBytes);
-            plan->grid = (int)G;
-            plan->ring = ring;
-            plan->span_cap = span;
-            plan->smem = fixed + (size_t)ring * kGemvRowBytes;
-            return QGEMM_OK;
-        }
-        if (G >= std::min<int64_t>(gmax, gcap)) break;
-    }
-    return QGEMM_ERR_UNSUPPORTED;
+    const int64_t G = std::min<int64_t>(std::min<int64_t>(U, gcap), sms);
+    const size_t fixed = gemv_fixed_smem(nb);
+    const size_t budget = (size_t)227 * 1024;
+    if (fixed + (size_t)kGemvMinRing * kGemvRowBytes > budget) return QGEMM_ERR_UNSUPPORTED;
+    const int ring = (int)std::min<size_t>(kGemvMaxRing, (budget - fixed) / kGemvRowBytes);
+    plan->grid = (int)G;
+    plan->ring = ring;
+    plan->span_cap = 0;
+    plan->smem = fixed + (size_t)ring * kGemvRowBytes;
+    return QGEMM_OK;
 }
 
 int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
@@ -184,7 +172,6 @@ int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     p.ng = gemv_groups(K);
     p.tiles = gemv_tiles(N);
     p.ring_rows = plan.ring;
-    p.span_cap = plan.span_cap;
 
     // launched as a programmatic dependent of xprep: starts streaming weights
     // while xprep runs and waits for it (griddepcontrol.wait) before reading x
