@@ -105,15 +105,18 @@ size_t qgemm_scale_bytes(int K, int N);
  * device.  Synchronises the device. Returns QGEMM_OK or QGEMM_ERR_CUDA. */
 int qgemm_device_error(int* h_code, int clear);
 
-/* Which kernel family qgemm() uses for M rows: 0 = split-K GEMV (CUDA-core
- * unpack + mma.sync), 1 = tcgen05 tensor-core GEMM with dequantisation into
- * shared memory. */
+/* Which kernel family qgemm() uses for M rows:
+ *   0 = split-K integer GEMV (M <= 4): activations rounded per (128-row group,
+ *       token) to int16 with a power-of-two scale, exact int32 dot products;
+ *   1 = split-K tensor-core GEMV (M <= 16): decoded fp16 codes in TMEM,
+ *       tcgen05.mma against the activations;
+ *   2 = tcgen05 tensor-core GEMM with dequantisation into shared memory. */
 int qgemm_path_for(int M, int K, int N);
 
 /* Launch plan qgemm() would use for this shape on the current device (or on a
  * 148-SM device when no GPU is visible).  out[0] = kernel family (as
  * qgemm_path_for), out[1] = grid size, out[2] = shared-memory ring rows (GEMV),
- * out[3] = activation-stage capacity in blocks (GEMV), out[4] = dynamic shared
+ * out[3] = CTAs resident per SM, out[4] = dynamic shared
  * memory bytes, out[5] = SM count used.  Host only; returns a qgemm_status. */
 int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out);
 
@@ -146,7 +149,11 @@ int qgemm_dequant(const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scale
  *   d_y      [M][N] fp16 output (RNE of the fp32 sum);
  *   d_ws     workspace of at least qgemm_workspace_bytes(M, K, N) bytes
  *            (may be NULL when that is 0).
- * M <= 16 runs the split-K GEMV, larger M the tcgen05 GEMM (qgemm_path_for). */
+ * M <= 16 runs a split-K GEMV, larger M the tcgen05 GEMM (qgemm_path_for).
+ * The integer GEMV (M <= 4) rounds each activation to the nearest multiple of
+ * 2^-e, 2^e being the power of two that brings the largest magnitude of its
+ * (128-row group, token) into [2^13, 2^14): an error of at most 2^-14 of that
+ * largest magnitude. */
 int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
           const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scales,
           const uint8_t* d_bits, const int32_t* d_offs,

@@ -134,7 +134,7 @@ def qgemm_path_for(M: int, K: int, N: int) -> int:
 def qgemm_plan_info(M: int, K: int, N: int, qw_rows: int) -> dict:
     out = (ctypes.c_int64 * 6)()
     _ok(_lib.qgemm_plan_info(M, K, N, int(qw_rows), out), "qgemm_plan_info")
-    return dict(path=out[0], grid=out[1], ring=out[2], span_cap=out[3], smem=out[4], sms=out[5])
+    return dict(path=out[0], grid=out[1], ring=out[2], ctas_per_sm=out[3], smem=out[4], sms=out[5])
 
 
 def qgemm_device_error(clear: bool = True) -> int:

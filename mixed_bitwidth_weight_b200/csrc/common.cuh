@@ -123,6 +123,18 @@ QG_DEV void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* 
         : "memory");
 }
 
+// 2D tensor copy global -> this CTA's shared memory of the box at (x, y) of
+// the tensor map (x in elements, a multiple of 16 bytes; y in rows), with an
+// L2 cache policy.  dst 128-byte aligned.  The whole box counts toward the
+// mbarrier's transaction bytes, out-of-range elements arriving as zeros.
+QG_DEV void tma_load_2d_hint(void* dst, const void* tmap, int x, int y, uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
 QG_DEV uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "gemv.cuh"
+#include "gemv_int.cuh"
 
 namespace {
 
@@ -19,6 +20,7 @@ constexpr int kVersion = 100;  // 0.1.0
 struct DeviceInfo {
     int sms = 0;
     bool gemv_attr[2] = {false, false};
+    bool int_attr[3] = {false, false, false};
 };
 
 DeviceInfo g_devs[64];
@@ -194,6 +196,174 @@ int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     return launch_status();
 }
 
+// ----------------------------------------------------------- integer GEMV
+constexpr int kPathGemvInt = 0, kPathGemvTc = 1, kPathGemm = 2;
+
+int int_mp(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
+int int_ctas_per_sm(int mp) { return mp <= 2 ? 2 : 1; }
+
+size_t int_fixed_smem(int nb, int mp) {
+    const size_t o = align_up((size_t)(nb + 1) * 4, 16) + 2 * kGemvSlots * 8 + 64 +
+                     (size_t)3 * kGemvTileCols * mp * 4;
+    return align_up(o, 1024);
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (the library does not link the driver library itself).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// Maps over qw [qw_rows][N] uint32 with boxes of 256 columns x 2^i rows.
+int make_int_maps(const uint32_t* qw, int64_t qw_rows, int N, IntMaps* maps) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return QGEMM_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)qw_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+    const cuuint32_t estr[2] = {1, 1};
+    for (int i = 0; i < kIntBoxMaps; ++i) {
+        const cuuint32_t box[2] = {(cuuint32_t)kGemvTileCols, (cuuint32_t)(1u << i)};
+        const CUresult r = fn(&maps->box[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qw), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return QGEMM_ERR_CUDA;
+    }
+    return QGEMM_OK;
+}
+
+// Workspace: [tickets][partial slots][activation records].
+struct IntWs {
+    size_t tickets, slots, rec, total;
+};
+
+IntWs int_ws_layout(int M, int K, int N, int sms) {
+    const int mp = int_mp(M);
+    const int nb = K / kBlockRows;
+    IntWs w;
+    w.tickets = 0;
+    w.slots = align_up((size_t)gemv_tiles(N) * 4, 256);
+    w.rec = w.slots + align_up((size_t)gemv_max_grid(K, N, sms) * 2 * mp * kGemvTileCols * 4, 256);
+    w.total = w.rec + align_up((size_t)(nb + 8) * int_rec_bytes(mp), 256);
+    return w;
+}
+
+// Two CTAs per SM for M <= 2 (one for M <= 4, whose activations need more
+// registers); grid capped as for the tensor-core GEMV so that every CTA's
+// range holds at least one unit.
+int plan_int(int M, int K, int N, int64_t qw_rows, int sms, GemvPlan* plan, int* cps_out) {
+    const int nb = K / kBlockRows;
+    const int mp = int_mp(M);
+    const int cps = int_ctas_per_sm(mp);
+    const int64_t U = (int64_t)gemv_tiles(N) * gemv_groups(K);
+    const int64_t C = (int64_t)gemv_tiles(N) * (qw_rows + gemv_groups(K));
+    const int64_t gcap = std::max<int64_t>(1, C / (8 * kGemvGroupBlocks + 2));
+    const int64_t G = std::min<int64_t>(std::min<int64_t>(U, gcap), (int64_t)cps * sms);
+    const size_t fixed = int_fixed_smem(nb, mp);
+    const size_t budget = (size_t)(cps == 2 ? 113 : 227) * 1024;
+    if (fixed + (size_t)kGemvMinRing * kIntRowBytes > budget) return QGEMM_ERR_UNSUPPORTED;
+    const int ring = (int)std::min<size_t>(kGemvMaxRing, (budget - fixed) / kIntRowBytes);
+    plan->grid = (int)G;
+    plan->ring = ring;
+    plan->span_cap = 0;
+    plan->smem = fixed + (size_t)ring * kIntRowBytes;
+    if (cps_out) *cps_out = cps;
+    return QGEMM_OK;
+}
+
+template <int MP>
+cudaError_t launch_int(const GemvPlan& plan, const IntParams& p, const IntMaps& maps, cudaStream_t stream,
+                       bool* attr_done) {
+    if (!*attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_int_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             227 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemv_int_kernel<MP>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        *attr_done = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.grid);
+    cfg.blockDim = dim3(kIntThreads);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemv_int_kernel<MP>, p, maps);
+}
+
+int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
+                 const uint16_t* scales, const uint8_t* bits, const int32_t* offs, int M, int K, int N,
+                 uint16_t* y, void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev) {
+    GemvPlan plan;
+    int st = plan_int(M, K, N, qw_rows, dev->sms, &plan, nullptr);
+    if (st != QGEMM_OK) return st;
+    const IntWs L = int_ws_layout(M, K, N, dev->sms);
+    if (ws_bytes < L.total || ws == nullptr) return QGEMM_ERR_WORKSPACE;
+    IntMaps maps;
+    if ((st = make_int_maps(qw, qw_rows, N, &maps)) != QGEMM_OK) return st;
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    const int nb = K / kBlockRows;
+    const int mp = int_mp(M);
+
+    IntPrepParams xp;
+    xp.x = x;
+    xp.perm = perm;
+    xp.bits = bits;
+    xp.rec = w8 + L.rec;
+    xp.M = M;
+    xp.K = K;
+    xp.nb = nb;
+    xp.mp = mp;
+    xp.x_bf16 = (x_dtype == QGEMM_BF16);
+    xprep_int_kernel<<<(nb + 7) / 8, 256, 0, stream>>>(xp);
+    if ((st = launch_status()) != QGEMM_OK) return st;
+
+    IntParams p;
+    p.rec = xp.rec;
+    p.qw = qw;
+    p.qw_rows = qw_rows;
+    p.scales = reinterpret_cast<const __half*>(scales);
+    p.bits = bits;
+    p.offs = offs;
+    p.y = reinterpret_cast<__half*>(y);
+    p.tickets = reinterpret_cast<int*>(w8 + L.tickets);
+    p.slots = reinterpret_cast<float*>(w8 + L.slots);
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.nb = nb;
+    p.ng = gemv_groups(K);
+    p.tiles = gemv_tiles(N);
+    p.ring_rows = plan.ring;
+    // programmatic dependent of xprep_int, as for the tensor-core GEMV
+    const cudaError_t e = (mp == 1)   ? launch_int<1>(plan, p, maps, stream, &dev->int_attr[0])
+                          : (mp == 2) ? launch_int<2>(plan, p, maps, stream, &dev->int_attr[1])
+                                      : launch_int<4>(plan, p, maps, stream, &dev->int_attr[2]);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return QGEMM_ERR_CUDA;
+    }
+    return launch_status();
+}
+
 }  // namespace
 
 // =========================================================== C ABI
@@ -265,14 +435,16 @@ size_t qgemm_scale_bytes(int K, int N) {
 int qgemm_path_for(int M, int K, int N) {
     (void)K;
     (void)N;
-    return M <= 16 ? 0 : 1;
+    return M <= kIntMaxM ? kPathGemvInt : M <= 16 ? kPathGemvTc : kPathGemm;
 }
 
 size_t qgemm_workspace_bytes(int M, int K, int N) {
     if (M <= 0 || check_shape(K, N) != QGEMM_OK) return 0;
     DeviceInfo* dev = nullptr;
     const int sms = (current_device_info(&dev) == QGEMM_OK) ? dev->sms : 148;
-    if (qgemm_path_for(M, K, N) == 0) return gemv_ws_layout(M, K, N, sms).total;
+    const int path = qgemm_path_for(M, K, N);
+    if (path == kPathGemvInt) return int_ws_layout(M, K, N, sms).total;
+    if (path == kPathGemvTc) return gemv_ws_layout(M, K, N, sms).total;
     return 0;
 }
 
@@ -287,12 +459,22 @@ int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out) {
     for (int i = 0; i < 6; ++i) out[i] = 0;
     out[0] = qgemm_path_for(M, K, N);
     out[5] = sms;
-    if (out[0] == 0) {
+    if (out[0] == kPathGemvInt) {
+        GemvPlan plan;
+        int cps = 1;
+        if ((st = plan_int(M, K, N, qw_rows, sms, &plan, &cps)) != QGEMM_OK) return st;
+        out[1] = plan.grid;
+        out[2] = plan.ring;
+        out[3] = cps;
+        out[4] = (int64_t)plan.smem;
+        return QGEMM_OK;
+    }
+    if (out[0] == kPathGemvTc) {
         GemvPlan plan;
         if ((st = plan_gemv(M, K, N, qw_rows, sms, &plan)) != QGEMM_OK) return st;
         out[1] = plan.grid;
         out[2] = plan.ring;
-        out[3] = plan.span_cap;
+        out[3] = 1;
         out[4] = (int64_t)plan.smem;
         return QGEMM_OK;
     }
@@ -353,7 +535,11 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm, const uint32_t* d
     DeviceInfo* dev = nullptr;
     if ((st = current_device_info(&dev)) != QGEMM_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (qgemm_path_for(M, K, N) == 0)
+    const int path = qgemm_path_for(M, K, N);
+    if (path == kPathGemvInt)
+        return run_gemv_int(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y,
+                            d_ws, ws_bytes, s, dev);
+    if (path == kPathGemvTc)
         return run_gemv(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y,
                         d_ws, ws_bytes, s, dev);
     return QGEMM_ERR_UNSUPPORTED;

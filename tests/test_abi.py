@@ -87,9 +87,11 @@ def test_workspace_and_sizes():
     assert lib.qgemm_packed_bytes(621, 28672) == 4 * 621 * 28672
     assert lib.qgemm_scale_bytes(8192, 28672) == 2 * 64 * 28672
     assert lib.qgemm_scale_bytes(160, 8) == 2 * 2 * 8
-    assert q.qgemm_path_for(1, 8192, 8192) == 0
-    assert q.qgemm_path_for(16, 8192, 8192) == 0
-    assert q.qgemm_path_for(2048, 8192, 8192) == 1
+    assert q.qgemm_path_for(1, 8192, 8192) == 0      # integer GEMV
+    assert q.qgemm_path_for(4, 8192, 8192) == 0
+    assert q.qgemm_path_for(5, 8192, 8192) == 1      # tensor-core GEMV
+    assert q.qgemm_path_for(16, 8192, 8192) == 1
+    assert q.qgemm_path_for(2048, 8192, 8192) == 2   # GEMM
 
 
 def _fake(addr):

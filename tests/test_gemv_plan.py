@@ -1,11 +1,11 @@
 """Host-side checks of the decode GEMV launch plan, without a GPU.
 
-The kernel splits the (256-column tile, 128-row group) units into contiguous,
-equal-cost ranges, one per CTA (see csrc/gemv.cuh).  This file replays that
+Both decode kernels (csrc/gemv_int.cuh for M <= 4, csrc/gemv.cuh for M <= 16)
+split the (256-column tile, 128-row group) units into contiguous, equal-cost
+ranges, one per CTA.  This file replays that
 split in Python for the workload shapes and checks what keeps the kernel in
 bounds: every unit is owned by exactly one CTA, the CTA that owns a unit is the
-one the reducer expects (cta_of), a CTA's blocks fit the activation stage the
-plan sized, a unit fits the shared-memory ring, and partial-sum slots stay
+one the reducer expects (cta_of), a unit fits the shared-memory ring, and partial-sum slots stay
 inside the workspace.
 """
 import bisect
@@ -58,7 +58,7 @@ def shapes():
     return out
 
 
-@pytest.mark.parametrize("M", [1, 4, 8, 9, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 9, 16])
 @pytest.mark.parametrize("case", shapes(), ids=lambda c: f"{c[0]}-{c[1]}x{c[2]}")
 def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     name, K, N, bits = case
@@ -67,18 +67,27 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     rows = int(offs[-1])
     tiles = (N + TILE - 1) // TILE
     plan = q.qgemm_plan_info(M, K, N, rows)
-    assert plan["path"] == 0
+    integer = M <= 4
+    assert plan["path"] == (0 if integer else 1)
     G = plan["grid"]
-    assert 1 <= G <= plan["sms"]                # one CTA per SM: each holds all of TMEM
-    assert plan["smem"] <= 227 * 1024
-    assert plan["ring"] >= 24
+    cps = plan["ctas_per_sm"]
+    if integer:
+        mp = 1 if M == 1 else 2 if M == 2 else 4
+        assert cps == (2 if mp <= 2 else 1)
+    else:
+        mp = 8 if M <= 8 else 16
+        assert cps == 1                          # each CTA holds all of TMEM
+    assert 1 <= G <= cps * plan["sms"]
+    # resident CTAs fit the SM's 228 KB (1 KB reserved per CTA)
+    assert cps * (plan["smem"] + 1024) <= 228 * 1024
+    assert plan["ring"] >= 80
     starts, cta_of, ng = replay(offs, tiles, G)
     assert starts[0] == 0 and starts[-1] == tiles * ng
     assert all(a <= b for a, b in zip(starts, starts[1:]))
-    mt = 1 if M <= 8 else 2
     ws = q.qgemm_workspace_bytes(M, K, N)
-    slot_bytes = mt * 8 * TILE * 4
-    act_bytes = nb * 64 * mt * 8 + ((nb + 3) // 4) * mt * 8 * 4 + 64
+    slot_bytes = mp * TILE * 4
+    rec = (72 * mp + 15) // 16 * 16 if integer else 64 * mp
+    act_bytes = nb * rec + (0 if integer else ((nb + 3) // 4) * mp * 4 + 64)
     assert ws >= ((tiles * 4 + 255) // 256 * 256) + G * 2 * slot_bytes + act_bytes
     rng = np.random.default_rng(K + N + M)
     for i in range(G):
@@ -94,7 +103,7 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
         expect = {c for c in range(first, last + 1) if starts[c] < starts[c + 1]}
         assert owners == expect, t
     # a unit (scale row, a group's word rows, activation records) fits the ring
-    rec = 64 * mt * 8
-    need = max(1 + int(offs[min(4 * g + 4, nb)] - offs[4 * g]) + -(-min(4, nb - 4 * g) * rec // 1056)
+    row_bytes = 1024 if integer else 1056
+    need = max(1 + int(offs[min(4 * g + 4, nb)] - offs[4 * g]) + -(-min(4, nb - 4 * g) * rec // row_bytes)
                for g in range(ng))
     assert need <= plan["ring"]

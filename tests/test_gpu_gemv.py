@@ -59,7 +59,7 @@ def test_dequant_bit_exact(q, K, N, kind):
 GEMV_SHAPES = [(32, 8), (160, 264), (1024, 1048), (2048, 4104), (4096, 776), (8192, 256)]
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 12, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 9, 12, 16])
 @pytest.mark.parametrize("K,N", GEMV_SHAPES)
 def test_gemv_parity(q, K, N, M):
     pr = P.make(K, N, M=M, kind="shuffled", seed=7 * M + K)
@@ -93,21 +93,66 @@ def test_gemv_bf16_large_and_tiny_activations(q):
     assert (y[1] == 0).all() or np.abs(y[1].float().cpu().numpy()).max() < 1e-3
 
 
+@pytest.mark.parametrize("M", [1, 4, 8])
 @pytest.mark.parametrize("kind", ["u2", "u3", "u4", "u5", "u6", "u8", "shuffled"])
-def test_gemv_one_hot_bit_exact(q, kind):
+def test_gemv_one_hot_bit_exact(q, kind, M):
+    """x = unit rows: y is a row of the fp16 dequantised matrix, exactly (both
+    GEMV families compute (q - z) * s exactly before the one rounding)."""
     K, N = 512, 520
-    pr = P.make(K, N, M=8, kind=kind, seed=17)
-    rng = np.random.default_rng(0)
-    js = rng.choice(K, size=8, replace=False)
-    x = torch.zeros(8, K, dtype=torch.float16)
-    x[np.arange(8), js] = 1.0
+    pr = P.make(K, N, M=M, kind=kind, seed=17)
+    rng = np.random.default_rng(M)
+    js = rng.choice(K, size=M, replace=False)
+    x = torch.zeros(M, K, dtype=torch.float16)
+    x[np.arange(M), js] = 1.0
     pr["x"] = x
     g = P.to_gpu(pr)
-    y = torch.empty((8, N), dtype=torch.float16, device="cuda")
-    q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, q.workspace(8, K, N))
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, q.workspace(M, K, N))
     w16 = oracle.dequant_f16(pr["qw"], pr["scales"].numpy(), pr["bits"], K)
     inv = np.argsort(pr["perm"])
     assert np.array_equal(y.cpu().numpy().view(np.uint16), w16[inv[js]])
+
+
+@pytest.mark.parametrize("M", [1, 2, 4])
+@pytest.mark.parametrize("x_dtype", [torch.float16, torch.bfloat16])
+def test_gemv_int_group_ranges_and_outliers(q, M, x_dtype):
+    """The integer GEMV scales activations per (128-row group, token): groups
+    whose magnitudes differ by 10^+-2 (fp16) or 10^+-3 (bf16), a group of
+    zeros and one 20x outlier per group must all stay within the output
+    tolerance."""
+    K, N = 2048, 776
+    pr = P.make(K, N, M=M, kind="shuffled", seed=31 + M, x_dtype=x_dtype)
+    x = pr["x"].double()
+    rng = np.random.default_rng(M)
+    ng = K // 128
+    span = 2 if x_dtype == torch.float16 else 3
+    gscale = torch.tensor(10.0 ** rng.uniform(-span, span, size=(M, ng)))
+    gscale[:, 3] = 0.0
+    inv = np.argsort(pr["perm"])                       # x column -> act-order row
+    grp = torch.as_tensor(inv // 128)
+    x = x * gscale[:, grp]
+    for m in range(M):
+        for gi in range(ng):
+            cols = np.nonzero(inv // 128 == gi)[0]
+            x[m, cols[rng.integers(len(cols))]] *= 20.0
+    pr["x"] = x.to(x_dtype)
+    assert bool(torch.isfinite(pr["x"].float()).all())
+    g = P.to_gpu(pr)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, q.workspace(M, K, N))
+    yr = P.ref_y(pr)
+    assert np.abs(yr).max() < 60000.0                  # the fp16 output does not overflow
+    P.check_close(y, yr)
+
+
+def test_gemv_zero_activations_give_zero(q):
+    K, N, M = 1024, 264, 2
+    pr = P.make(K, N, M=M, kind="shuffled", seed=3)
+    pr["x"] = torch.zeros(M, K, dtype=torch.float16)
+    g = P.to_gpu(pr)
+    y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, q.workspace(M, K, N))
+    assert bool((y == 0).all())
 
 
 def test_gemv_deterministic_and_workspace_reset(q):
