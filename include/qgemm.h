@@ -160,6 +160,42 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
           int M, int K, int N, uint16_t* d_y,
           void* d_ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------- allocation-free decode
+ * The paper has no counterpart to this entry point; it serves callers that
+ * cannot allocate device memory.  qgemm() needs a caller-provided workspace,
+ * and some callers have no way to get one: a runtime that plans every byte of
+ * device memory up front and owns the only allocator, a plugin that is not
+ * allowed to allocate behind its host's back, or a latency-bound decode loop
+ * that cannot afford cudaMalloc/cudaFree (cudaFree synchronises the device).
+ *
+ * qgemm_decode_noalloc computes exactly what qgemm() computes for M <= 4 (the
+ * integer decode GEMV, same kernels and same split, so the same result) but
+ * takes its scratch from a buffer of QGEMM_NOALLOC_SCRATCH_BYTES built into
+ * the library.  Every GPU that loads the library holds that buffer until the
+ * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *
+ *   Arguments, layouts and ownership as qgemm(), without d_ws / ws_bytes.
+ *   Limits: 1 <= M <= 4 (QGEMM_ERR_SHAPE otherwise); a shape whose scratch
+ *     (qgemm_workspace_bytes(M, K, N)) exceeds QGEMM_NOALLOC_SCRATCH_BYTES is
+ *     refused with QGEMM_ERR_WORKSPACE before anything is launched.
+ *   First call on a device: looks up the buffer's device address
+ *     (cudaGetSymbolAddress, with that device current) and sets the kernels'
+ *     shared-memory attributes; make this first call before any stream
+ *     capture.
+ *   Shared state: every call on a device uses the same buffer.  Each call
+ *     first zeroes, on its stream, the part that must start at zero (the
+ *     per-tile tickets); the rest is overwritten before it is read.  Calls
+ *     that overlap on the GPU (other streams, other threads) race on the
+ *     buffer and give wrong results: order them, e.g. on one stream.
+ *   Returns a qgemm_status as qgemm(). */
+#define QGEMM_NOALLOC_SCRATCH_BYTES ((size_t)6 << 20)
+
+int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm,
+                         const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scales,
+                         const uint8_t* d_bits, const int32_t* d_offs,
+                         int M, int K, int N, uint16_t* d_y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -54,6 +54,7 @@ def _load():
         "qgemm_pack": (I, [P, P, P, I, I, I64, P, P]),
         "qgemm_dequant": (I, [P, I64, P, P, P, I, I, P, P]),
         "qgemm": (I, [P, I, P, P, I64, P, P, P, I, I, I, P, P, SZ, P]),
+        "qgemm_decode_noalloc": (I, [P, I, P, P, I64, P, P, P, I, I, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -187,6 +188,31 @@ def qgemm(x, perm, qw, scales, bits, offs, y, ws=None, stream=None):
                    _dev(scales, torch.float16, "scales"), _dev(bits, torch.uint8, "bits"),
                    _dev(offs, torch.int32, "offs"), M, K, N, _dev(y, torch.float16, "y"),
                    wsp, wsb, _stream(stream)), "qgemm")
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 6 << 20
+
+
+def qgemm_decode_noalloc(x, perm, qw, scales, bits, offs, y, stream=None):
+    """As qgemm() for M <= 4, with no workspace: the scratch is a buffer built
+    into the library, so nothing is allocated (for callers that cannot
+    allocate device memory).  Calls that overlap on the GPU race on that
+    buffer; the first call on a device should come before any stream capture."""
+    import torch
+    M, K = x.shape
+    N = y.shape[1]
+    if x.dtype == torch.float16:
+        xdt = QGEMM_F16
+    elif x.dtype == torch.bfloat16:
+        xdt = QGEMM_BF16
+    else:
+        raise TypeError("x must be float16 or bfloat16")
+    _ok(_lib.qgemm_decode_noalloc(_dev(x, None, "x"), xdt, _dev(perm, torch.int32, "perm"),
+                                  _dev(qw, (torch.int32, torch.uint32), "qw"), qw.shape[0],
+                                  _dev(scales, torch.float16, "scales"), _dev(bits, torch.uint8, "bits"),
+                                  _dev(offs, torch.int32, "offs"), M, K, N, _dev(y, torch.float16, "y"),
+                                  _stream(stream)), "qgemm_decode_noalloc")
     return y
 
 

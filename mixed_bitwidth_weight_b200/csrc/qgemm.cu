@@ -364,6 +364,34 @@ int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t
     return launch_status();
 }
 
+// ------------------------------------------------ allocation-free decode
+// Scratch of qgemm_decode_noalloc, built into the library so that the call
+// allocates nothing.  Zero-initialised at module load; every call re-zeroes
+// the tickets it needs at zero.  In host code `g_noalloc_scratch` names a
+// host-side stand-in, not device memory: kernels get the address that
+// cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QGEMM_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[64];
+std::mutex g_noalloc_mu;
+
+// Device address of the buffer on the current device, looked up once per device.
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QGEMM_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return QGEMM_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return QGEMM_OK;
+}
+
 }  // namespace
 
 // =========================================================== C ABI
@@ -543,6 +571,33 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm, const uint32_t* d
         return run_gemv(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y,
                         d_ws, ws_bytes, s, dev);
     return QGEMM_ERR_UNSUPPORTED;
+}
+
+int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm, const uint32_t* d_qw,
+                         int64_t qw_rows, const uint16_t* d_scales, const uint8_t* d_bits,
+                         const int32_t* d_offs, int M, int K, int N, uint16_t* d_y, void* stream) {
+    if (!d_x || !d_perm || !d_qw || !d_scales || !d_bits || !d_offs || !d_y) return QGEMM_ERR_NULL;
+    if (x_dtype != QGEMM_F16 && x_dtype != QGEMM_BF16) return QGEMM_ERR_DTYPE;
+    int st = check_shape(K, N);
+    if (st != QGEMM_OK) return st;
+    if (M < 1 || M > kIntMaxM) return QGEMM_ERR_SHAPE;
+    if ((st = check_rows(K, qw_rows)) != QGEMM_OK) return st;
+    if (!aligned16(d_x) || !aligned16(d_perm) || !aligned16(d_qw) || !aligned16(d_scales) || !aligned16(d_y))
+        return QGEMM_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    if ((st = current_device_info(&dev)) != QGEMM_OK) return st;
+    const IntWs L = int_ws_layout(M, K, N, dev->sms);
+    if (L.total > QGEMM_NOALLOC_SCRATCH_BYTES) return QGEMM_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != QGEMM_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the tickets (the layout's first bytes, up to the partial-sum slots) must start at zero
+    if (cudaMemsetAsync(scratch, 0, L.slots, s) != cudaSuccess) {
+        cudaGetLastError();
+        return QGEMM_ERR_CUDA;
+    }
+    return run_gemv_int(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y, scratch,
+                        QGEMM_NOALLOC_SCRATCH_BYTES, s, dev);
 }
 
 }  // extern "C"
