@@ -1,0 +1,394 @@
+// Prefill GEMM on the 5th-generation tensor cores: y = x[:, perm] . dequant(Wq)
+// for M > 16 (the quantised GEMM of the exllamav2 report, "解法哲学", which
+// the pages credit with near-bandwidth decode and tensor-core prefill).
+//
+// Two kernels:
+// * xperm_kernel writes x_p = x[:, perm] (the act-order gather) into the
+//   workspace as fp16, so that the activation tiles are plain 2D boxes and
+//   both MMA operands are fp16 (bf16 input is scaled per row by a power of
+//   two first, exactly, and y is scaled back).
+// * gemm_kernel computes one 256 x 256 tile of y per CTA.  Warp roles:
+//     warp 0     - TMA producer: activation tiles (256 rows x 64 k, 128-byte
+//                  swizzle) and, per 64-row k step, the step's word rows
+//                  (2D boxes) and its group's scale row;
+//     warp 1     - allocates TMEM (two 128 x 256 fp32 accumulators, all 512
+//                  columns) and issues the MMAs from one thread:
+//                  tcgen05.mma kind::f16, M = 128, N = 256, K = 16, both
+//                  operands from shared memory;
+//     warps 2-9  - dequantise: thread n decodes the 64 codes of column n in
+//                  the step (two 32-row blocks, each at its own width), forms
+//                  w = (q - 2^(b-1)) * s exactly in fp32, rounds once to fp16
+//                  (the bit-exact dequantised weight) and writes row n of the B tile in the
+//                  K-major 128-byte-swizzled layout the MMA reads; after the
+//                  last step they move the accumulators TMEM -> fp16 y.
+// Every wait is bounded; a timeout sets the device error word, the CTA skips
+// the remaining work, waits for its copies and MMAs and frees TMEM.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "pack_dequant.cuh"
+
+namespace qg {
+
+constexpr int kGemmBM = 256;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBK = 64;                              // two 32-row blocks per k step
+constexpr int kGemmAStages = 3;
+constexpr int kGemmBStages = 2;
+constexpr int kGemmRStages = 3;
+constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;       // 32 KB
+constexpr int kGemmBBytes = kGemmBN * kGemmBK * 2;       // 32 KB
+constexpr int kGemmRawRows = 16;                         // word rows of two blocks, at most
+constexpr int kGemmRBytes = (kGemmRawRows + 1) * 1024;   // scale row + word rows
+constexpr int kGemmDecWarps = 8;
+constexpr int kGemmThreads = 64 + kGemmDecWarps * 32;
+constexpr int kGemmBoxMaps = 5;                          // word boxes of 1, 2, 4, 8, 16 rows
+constexpr int kGemmFixedSmem =
+    kGemmAStages * kGemmABytes + kGemmBStages * kGemmBBytes + kGemmRStages * kGemmRBytes + 1024;
+
+struct GemmMaps {
+    CUtensorMap a;                    // x_p [M][K], box {64, 256}, 128-byte swizzle
+    CUtensorMap w[kGemmBoxMaps];      // qw [qw_rows][N], box {256, 2^i}
+};
+
+struct GemmParams {
+    const int* xshift;   // [M] row shifts of bf16 input (x_bf16 != 0)
+    const __half* scales;
+    const uint8_t* bits;
+    const int32_t* offs;
+    int64_t qw_rows;
+    __half* y;
+    int M, K, N, nb, mtiles, x_bf16;
+};
+
+struct XpermParams {
+    const uint16_t* x;
+    const int32_t* perm;
+    uint16_t* xp;
+    int* xshift;   // [M] per-row power-of-two shift (bf16 input)
+    int M, K, x_bf16;
+};
+
+// x_p[m][k] = fp16(x[m][perm[k]] * 2^-shift[m]), one CTA per row, 8 k per
+// thread step (16-byte stores).  fp16 input: shift 0, a plain gather.  bf16
+// input: shift puts the row's largest magnitude in [2^14, 2^15), so the
+// conversion to fp16 is exact for every value within 2^24 of the maximum;
+// the GEMM multiplies the row of y by 2^shift.
+__global__ void __launch_bounds__(256) xperm_kernel(const XpermParams p) {
+    __shared__ int s_e[8];
+    const int64_t m = blockIdx.x;
+    const uint16_t* row = p.x + m * p.K;
+    int shift = 0;
+    if (p.x_bf16) {
+        int e = 0;
+        for (int k = threadIdx.x; k < p.K; k += blockDim.x) e = max(e, (int)((row[k] >> 7) & 0xFF));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+        if ((threadIdx.x & 31) == 0) s_e[threadIdx.x >> 5] = e;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            int v = threadIdx.x < 8 ? s_e[threadIdx.x] : 0;
+#pragma unroll
+            for (int o = 4; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (threadIdx.x == 0) s_e[0] = v;
+        }
+        __syncthreads();
+        shift = (s_e[0] == 0) ? 0 : s_e[0] - 141;  // max < 2^(E-126); 2^(E-127-shift) = 2^14
+        if (threadIdx.x == 0) p.xshift[m] = shift;
+    }
+    const int s1 = shift / 2, s2 = shift - shift / 2;  // 2^-shift as two normal factors
+    const float f1 = __int_as_float((127 - s1) << 23), f2 = __int_as_float((127 - s2) << 23);
+    for (int k0 = threadIdx.x * 8; k0 < p.K; k0 += blockDim.x * 8) {
+        const int4 i0 = *reinterpret_cast<const int4*>(p.perm + k0);
+        const int4 i1 = *reinterpret_cast<const int4*>(p.perm + k0 + 4);
+        const int idx[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+        uint32_t v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            uint16_t h[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int a = idx[2 * u + t];
+                uint16_t raw = 0;
+                if ((unsigned)a < (unsigned)p.K) raw = row[a];
+                else set_dev_error(QGEMM_DEV_BAD_PERM);
+                if (p.x_bf16) {
+                    const float f = __uint_as_float((uint32_t)raw << 16) * f1 * f2;
+                    h[t] = __half_as_ushort(__float2half_rn(f));
+                } else {
+                    h[t] = raw;
+                }
+            }
+            v[u] = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+        }
+        *reinterpret_cast<uint4*>(p.xp + m * p.K + k0) = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+}
+
+QG_DEV void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Two fp32 values -> one 32-bit pair of the activation type, RNE; lo in the
+// low half.
+template <bool BF16>
+QG_DEV uint32_t pack2(float lo, float hi) {
+    uint32_t d;
+    if constexpr (BF16) asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    else asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// The 32 codes of one block for this thread's column, dequantised:
+// out[i] = pair (w[2i], w[2i+1]).  w0 = word row 0 of the block at this column,
+// word rows 1 KB apart.  (2^23 + q) - (2^23 + z) = q - z exactly, and (q - z) * s
+// has at most 19 significant bits, so the one rounding is the cvt.
+template <int B, bool BF16>
+QG_DEV void dequant_block32(const uint8_t* w0, float s, uint32_t (&out)[16]) {
+    constexpr uint32_t mask = (1u << B) - 1u;
+    const float zoff = 8388608.f + (float)(1 << (B - 1));
+    uint32_t w[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) w[i] = *reinterpret_cast<const uint32_t*>(w0 + i * 1024);
+#pragma unroll
+    for (int r = 0; r < 32; r += 2) {
+        float f[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int bit = (r + u) * B, wi = bit >> 5, sh = bit & 31;
+            uint32_t q;
+            if (sh + B <= 32) q = (w[wi] >> sh) & mask;
+            else q = __funnelshift_r(w[wi], w[wi + 1 < B ? wi + 1 : wi], sh) & mask;
+            f[u] = (__uint_as_float(0x4B000000u | q) - zoff) * s;
+        }
+        out[r / 2] = pack2<BF16>(f[0], f[1]);
+    }
+}
+
+template <bool BF16>
+QG_DEV void dequant_block32_any(int b, const uint8_t* w0, float s, uint32_t (&out)[16]) {
+    switch (b) {
+        case 2: dequant_block32<2, BF16>(w0, s, out); break;
+        case 3: dequant_block32<3, BF16>(w0, s, out); break;
+        case 4: dequant_block32<4, BF16>(w0, s, out); break;
+        case 5: dequant_block32<5, BF16>(w0, s, out); break;
+        case 6: dequant_block32<6, BF16>(w0, s, out); break;
+        default: dequant_block32<8, BF16>(w0, s, out); break;
+    }
+}
+
+// kind::f16 instruction descriptor: fp32 D, A and B both fp16 or both bf16,
+// both K-major.
+QG_DEV constexpr uint32_t idesc_kf16(int M, int N, bool bf16) {
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_kernel(const GemmParams p, const __grid_constant__ GemmMaps maps) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nb = p.nb;
+    // 1024-byte aligned operand buffers (the swizzle pattern is address based)
+    uint8_t* base = smem + ((1024 - (smem_u32(smem) & 1023)) & 1023);
+    uint8_t* sA = base;
+    uint8_t* sB = sA + kGemmAStages * kGemmABytes;
+    uint8_t* sR = sB + kGemmBStages * kGemmBBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sR + kGemmRStages * kGemmRBytes);
+    uint64_t* a_full = bars;
+    uint64_t* a_empty = a_full + kGemmAStages;
+    uint64_t* b_full = a_empty + kGemmAStages;
+    uint64_t* b_empty = b_full + kGemmBStages;
+    uint64_t* r_full = b_empty + kGemmBStages;
+    uint64_t* r_empty = r_full + kGemmRStages;
+    uint64_t* acc_full = r_empty + kGemmRStages;
+    int* s_misc = reinterpret_cast<int*>(acc_full + 1);  // [0] bad schedule, [1] abort, [2] tmem base
+    int32_t* s_offs = s_misc + 8;
+
+    const int mt = blockIdx.x % p.mtiles, ntile = blockIdx.x / p.mtiles;
+    const int m0 = mt * kGemmBM, n0 = ntile * kGemmBN;
+    const int nk = (p.K + kGemmBK - 1) / kGemmBK;
+
+    // ---- schedule into shared memory, validated before any weight access
+    if (tid < 8) s_misc[tid] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int j = tid; j <= nb; j += kGemmThreads) {
+        const int o = p.offs[j];
+        s_offs[j] = o;
+        if (j < nb) {
+            const int b = p.bits[j];
+            if (!width_ok(b) || p.offs[j + 1] - o != b) bad = true;
+        }
+    }
+    if (tid == 0 && (p.offs[0] != 0 || (int64_t)p.offs[nb] != p.qw_rows)) bad = true;
+    if (bad) atomicOr(&s_misc[0], 1);
+    if (tid == 0) {
+        for (int i = 0; i < kGemmAStages; ++i) {
+            mbar_init(&a_full[i], 1);
+            mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < kGemmBStages; ++i) {
+            mbar_init(&b_full[i], kGemmDecWarps);
+            mbar_init(&b_empty[i], 1);
+        }
+        for (int i = 0; i < kGemmRStages; ++i) {
+            mbar_init(&r_full[i], 1);
+            mbar_init(&r_empty[i], kGemmDecWarps);
+        }
+        mbar_init(acc_full, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(reinterpret_cast<uint32_t*>(&s_misc[2]), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)s_misc[2];
+    if (s_misc[0]) {
+        if (tid == 0) set_dev_error(QGEMM_DEV_BAD_SCHEDULE);
+    } else if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            int i = 0;
+            bool ok = true;
+            for (; i < nk; ++i) {
+                const int sa = i % kGemmAStages, sr = i % kGemmRStages;
+                if ((i >= kGemmAStages && !mbar_wait(&a_empty[sa], (uint32_t)(((i / kGemmAStages) - 1) & 1))) ||
+                    (i >= kGemmRStages && !mbar_wait(&r_empty[sr], (uint32_t)(((i / kGemmRStages) - 1) & 1)))) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&a_full[sa], (uint32_t)kGemmABytes);
+                tma_load_2d(sA + sa * kGemmABytes, &maps.a, i * kGemmBK, m0, &a_full[sa]);
+                const int j0 = 2 * i, j1 = min(j0 + 2, nb);
+                const int r0 = s_offs[j0], rows = s_offs[j1] - r0;
+                const int g = (i * kGemmBK) / 128;
+                const int cols = min(kGemmBN, p.N - n0);
+                uint8_t* dst = sR + sr * kGemmRBytes;
+                mbar_arrive_expect_tx(&r_full[sr], (uint32_t)(cols * 2 + rows * 1024));
+                bulk_g2s(dst, p.scales + (size_t)g * p.N + n0, (uint32_t)cols * 2, &r_full[sr]);
+                int r = 0;
+#pragma unroll 1
+                for (int bx = kGemmBoxMaps - 1; bx >= 0; --bx)
+                    if (rows & (1 << bx)) {
+                        tma_load_2d(dst + (size_t)(1 + r) * 1024, &maps.w[bx], n0, r0 + r, &r_full[sr]);
+                        r += 1 << bx;
+                    }
+            }
+            if (!ok) {  // let every issued copy land before the CTA can exit
+                s_misc[1] = 1;
+                for (int k = max(0, i - kGemmAStages); k < i; ++k)
+                    mbar_wait(&a_full[k % kGemmAStages], (uint32_t)((k / kGemmAStages) & 1));
+                for (int k = max(0, i - kGemmRStages); k < i; ++k)
+                    mbar_wait(&r_full[k % kGemmRStages], (uint32_t)((k / kGemmRStages) & 1));
+            }
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = idesc_kf16(128, kGemmBN, BF16);
+            for (int i = 0; i < nk && !s_misc[1]; ++i) {
+                const int sa = i % kGemmAStages, sb = i % kGemmBStages;
+                if (!mbar_wait(&a_full[sa], (uint32_t)((i / kGemmAStages) & 1)) ||
+                    !mbar_wait(&b_full[sb], (uint32_t)((i / kGemmBStages) & 1))) {
+                    s_misc[1] = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(sA + sa * kGemmABytes), b_addr = smem_u32(sB + sb * kGemmBBytes);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+                        const uint64_t ad = smem_desc(a_addr + h * (128 * 128) + kk * 32, 16, 1024, 2);
+                        const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024, 2);
+                        tc_mma_ss(tmem + h * kGemmBN, ad, bd, kIdesc, (i | kk) != 0);
+                    }
+                tc_commit(&a_empty[sa]);
+                tc_commit(&b_empty[sb]);
+            }
+            tc_commit(acc_full);  // also when aborted: completes once issued MMAs are done
+        }
+    } else {
+        // ================================================= dequant warps
+        const int n = tid - 64;                 // column within the tile
+        for (int i = 0; i < nk; ++i) {
+            const int sr = i % kGemmRStages, sb = i % kGemmBStages;
+            if (s_misc[1] || !mbar_wait(&r_full[sr], (uint32_t)((i / kGemmRStages) & 1)) ||
+                (i >= kGemmBStages && !mbar_wait(&b_empty[sb], (uint32_t)(((i / kGemmBStages) - 1) & 1)))) {
+                s_misc[1] = 1;
+                break;
+            }
+            const uint8_t* raw = sR + sr * kGemmRBytes;
+            const float s = __half2float(reinterpret_cast<const __half*>(raw)[n]);
+            uint8_t* brow = sB + sb * kGemmBBytes + n * 128;
+            const int j0 = 2 * i;
+            const int r0 = s_offs[j0];
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk) {
+                const int j = j0 + blk;
+                uint32_t out[16];
+                if (j < nb) {
+                    dequant_block32_any<BF16>(s_offs[j + 1] - s_offs[j],
+                                              raw + 1024 + (size_t)(s_offs[j] - r0) * 1024 + n * 4, s, out);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) out[u] = 0;
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int chunk = 4 * blk + c;
+                    *reinterpret_cast<uint4*>(brow + ((chunk ^ (n & 7)) << 4)) =
+                        make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&b_full[sb]);
+                mbar_arrive(&r_empty[sr]);
+            }
+        }
+        // ---- epilogue: TMEM -> y (fp16)
+        const bool ok = mbar_wait(acc_full, 0) && !s_misc[1];
+        tc_fence_after();
+        if (ok) {
+            const int q = warp & 3, h = (warp - 2) >> 2;
+            const int row = m0 + h * 128 + q * 32 + lane;
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + h * kGemmBN;
+            const int sh = (p.x_bf16 && row < p.M) ? p.xshift[row] : 0;
+            const float g1 = __int_as_float((127 + sh / 2) << 23), g2 = __int_as_float((127 + (sh - sh / 2)) << 23);
+#pragma unroll 1
+            for (int c = 0; c < kGemmBN; c += 16) {
+                float v[16];
+                tmem_ld16(taddr + c, v);
+                if (row < p.M && n0 + c < p.N) {
+                    uint32_t hv[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const __half2 t = __floats2half2_rn(v[2 * u] * g1 * g2, v[2 * u + 1] * g1 * g2);
+                        hv[u] = *reinterpret_cast<const uint32_t*>(&t);
+                    }
+                    __half* dst = p.y + (size_t)row * p.N + n0 + c;
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                    if (n0 + c + 8 < p.N) *reinterpret_cast<uint4*>(dst + 8) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace qg

@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "gemv.cuh"
 #include "gemv_int.cuh"
+#include "gemm.cuh"
 
 namespace {
 
@@ -21,6 +22,7 @@ struct DeviceInfo {
     int sms = 0;
     bool gemv_attr[2] = {false, false};
     bool int_attr[3] = {false, false, false};
+    bool gemm_attr[2] = {false, false};
 };
 
 DeviceInfo g_devs[64];
@@ -364,6 +366,90 @@ int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t
     return launch_status();
 }
 
+// ------------------------------------------------------------------ GEMM
+int gemm_mtiles(int M) { return (M + kGemmBM - 1) / kGemmBM; }
+int gemm_ntiles(int N) { return (N + kGemmBN - 1) / kGemmBN; }
+// Workspace: [x_p fp16 M x K][row shifts int32 M].
+size_t gemm_ws_xshift(int M, int K) { return align_up((size_t)M * K * 2, 256); }
+size_t gemm_ws_bytes(int M, int K) { return gemm_ws_xshift(M, K) + align_up((size_t)M * 4, 256); }
+size_t gemm_smem(int nb) { return (size_t)kGemmFixedSmem + 512 + (size_t)(nb + 1) * 4; }
+
+int make_gemm_maps(const void* xp, int x_dtype, int M, int K, const uint32_t* qw, int64_t qw_rows, int N,
+                   GemmMaps* maps) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return QGEMM_ERR_CUDA;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)kGemmBM};
+        const cuuint32_t estr[2] = {1, 1};
+        (void)x_dtype;  // x_p is fp16 for both input types
+        const CUresult r = fn(&maps->a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(xp), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return QGEMM_ERR_CUDA;
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)qw_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+    const cuuint32_t estr[2] = {1, 1};
+    for (int i = 0; i < kGemmBoxMaps; ++i) {
+        const cuuint32_t box[2] = {(cuuint32_t)kGemmBN, (cuuint32_t)(1u << i)};
+        const CUresult r = fn(&maps->w[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qw), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return QGEMM_ERR_CUDA;
+    }
+    return QGEMM_OK;
+}
+
+int run_gemm(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
+             const uint16_t* scales, const uint8_t* bits, const int32_t* offs, int M, int K, int N, uint16_t* y,
+             void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev) {
+    if (ws == nullptr || ws_bytes < gemm_ws_bytes(M, K)) return QGEMM_ERR_WORKSPACE;
+    const int nb = K / kBlockRows;
+    const size_t smem = gemm_smem(nb);
+    if (smem > (size_t)227 * 1024) return QGEMM_ERR_UNSUPPORTED;
+    const bool bf16 = (x_dtype == QGEMM_BF16);
+    if (!dev->gemm_attr[0]) {
+        if (cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess)
+            return QGEMM_ERR_CUDA;
+        dev->gemm_attr[0] = true;
+    }
+    int* xshift = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + gemm_ws_xshift(M, K));
+    GemmMaps maps;
+    int st = make_gemm_maps(ws, x_dtype, M, K, qw, qw_rows, N, &maps);
+    if (st != QGEMM_OK) return st;
+
+    XpermParams xq;
+    xq.x = static_cast<const uint16_t*>(x);
+    xq.perm = perm;
+    xq.xp = static_cast<uint16_t*>(ws);
+    xq.xshift = xshift;
+    xq.M = M;
+    xq.K = K;
+    xq.x_bf16 = bf16;
+    xperm_kernel<<<(unsigned)M, 256, 0, stream>>>(xq);
+    if ((st = launch_status()) != QGEMM_OK) return st;
+
+    GemmParams p;
+    p.xshift = xshift;
+    p.scales = reinterpret_cast<const __half*>(scales);
+    p.bits = bits;
+    p.offs = offs;
+    p.qw_rows = qw_rows;
+    p.y = reinterpret_cast<__half*>(y);
+    p.M = M;
+    p.K = K;
+    p.N = N;
+    p.nb = nb;
+    p.mtiles = gemm_mtiles(M);
+    p.x_bf16 = bf16;
+    const unsigned grid = (unsigned)((int64_t)gemm_mtiles(M) * gemm_ntiles(N));
+    gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(p, maps);
+    return launch_status();
+}
+
 // ------------------------------------------------ allocation-free decode
 // Scratch of qgemm_decode_noalloc, built into the library so that the call
 // allocates nothing.  Zero-initialised at module load; every call re-zeroes
@@ -473,7 +559,7 @@ size_t qgemm_workspace_bytes(int M, int K, int N) {
     const int path = qgemm_path_for(M, K, N);
     if (path == kPathGemvInt) return int_ws_layout(M, K, N, sms).total;
     if (path == kPathGemvTc) return gemv_ws_layout(M, K, N, sms).total;
-    return 0;
+    return gemm_ws_bytes(M, K);
 }
 
 int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out) {
@@ -504,6 +590,13 @@ int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out) {
         out[2] = plan.ring;
         out[3] = 1;
         out[4] = (int64_t)plan.smem;
+        return QGEMM_OK;
+    }
+    if (out[0] == kPathGemm) {
+        out[1] = (int64_t)gemm_mtiles(M) * gemm_ntiles(N);
+        out[2] = 0;
+        out[3] = 1;
+        out[4] = (int64_t)gemm_smem(K / kBlockRows);
         return QGEMM_OK;
     }
     return QGEMM_ERR_UNSUPPORTED;
@@ -570,6 +663,9 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm, const uint32_t* d
     if (path == kPathGemvTc)
         return run_gemv(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y,
                         d_ws, ws_bytes, s, dev);
+    if (path == kPathGemm)
+        return run_gemm(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y, d_ws,
+                        ws_bytes, s, dev);
     return QGEMM_ERR_UNSUPPORTED;
 }
 

@@ -122,3 +122,15 @@ def test_host_argument_errors_return_status_without_launching():
     assert lib.qgemm_pack(_fake(0), _fake(A), _fake(A), 128, 64, 16, _fake(A), _fake(0)) == -1
     assert lib.qgemm_pack(_fake(A), _fake(A), _fake(A), 128, 64, 16, _fake(A + 2), _fake(0)) == -4
     assert lib.qgemm_dequant(_fake(A), 16, _fake(A), _fake(A), _fake(A), 100, 64, _fake(A), _fake(0)) == -2
+
+
+def test_gemm_plan_and_workspace():
+    """M > 16: one 256 x 256 output tile per CTA, the permuted activations in
+    the workspace, shared memory within the 227 KB a CTA may use up to K = 65536."""
+    plan = q.qgemm_plan_info(2048, 8192, 28672, 992)
+    assert plan["path"] == 2
+    assert plan["grid"] == 8 * 112
+    assert plan["smem"] <= 227 * 1024
+    assert q.qgemm_workspace_bytes(2048, 8192, 28672) >= 2048 * 8192 * 2
+    big = q.qgemm_plan_info(17, 65536, 8, 2 * 2048)
+    assert big["smem"] <= 227 * 1024 and big["grid"] == 1
