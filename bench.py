@@ -16,8 +16,11 @@ Extra objects on the same line:
   cpu_baseline  the CPU oracle timed on the host cores (rank 0, N = 1);
   e2e           the same metric through the public call with host buffers
                 (x copied in from pinned memory, y copied back, every step);
-  sweep         other M of the same shape (GB/s), and the 80-layer Llama-3-70B
-                linear stack as tokens/s, when --full is given;
+  prefill       TFLOP/s of the M = 2048 prefill GEMM (K = 8192, N = 28672,
+                4.0 bpw, bf16 activations) against the dense tensor peak;
+  decode_m_gbs, crossover_sweep, stack (with --full): other M of the headline
+                shape, the 8192 x 8192 M sweep that locates the GEMV/GEMM
+                crossover, and the 80-layer Llama-3-70B linear stack as tokens/s;
   clocks        SM clocks and throttle reasons sampled during the timed region.
 
 --impl reference times the CPU oracle (the only reference implementation this
@@ -45,6 +48,11 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 HEADLINE = "decode_8192x28672_2p55"
+PREFILL = "prefill_2048x8192x28672_4p0"
+PREFILL_M = 2048
+SWEEP = "sweep_8192x8192_3p75"
+SWEEP_MS = (1, 2, 4, 8, 16, 32, 64, 128, 256, 512)
+STACK = "llama70b_stack_2p5"
 METRIC = "Q-GEMM weight GB/s at M=1 (% of HBM) and TFLOP/s at M=2048 (% of peak)"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
@@ -273,6 +281,81 @@ def bench_decode(q, w, M, steps, warmup, ws, chunk=192):
                 gbs=nbytes * steps / secs / 1e9, us=secs / steps * 1e6, layer=base)
 
 
+def bench_prefill(q, w, M, steps, warmup, ws):
+    """TFLOP/s of the prefill GEMM, rotating over weight copies > 3x L2."""
+    base = Layer(w, M)
+    one = 4 * base.N * base.rows + 2 * ((base.K + 127) // 128) * base.N
+    R = max(1, math.ceil((3 * L2_BYTES + 1) / one))
+    layers = [base]
+    for r in range(1, R):
+        L = Layer.__new__(Layer)
+        L.__dict__.update(base.__dict__)
+        L.qw = base.qw.clone()
+        L.scales = base.scales.clone()
+        layers.append(L)
+    fn = lambda i: layers[i % R].call(q)  # noqa: E731
+    wg = run_steps(fn, warmup, 16)
+    tg = run_steps(fn, steps, 16)
+    for g in wg:
+        g.replay()
+    secs, t0, t1 = time_graphs(tg, ws)
+    secs = max_over_ranks(secs, ws)
+    flops = 2.0 * M * base.K * base.N
+    return dict(secs=secs, t0=t0, t1=t1, flops=flops, rows=base.rows, copies=R,
+                tflops=flops * steps / secs / 1e12, ms=secs / steps * 1e3, layer=base)
+
+
+def bench_sweep(q, w, Ms, ws):
+    """Crossover sweep: one shape, several M; GB/s and TFLOP/s per M and the path used."""
+    out = {}
+    for M in Ms:
+        base = Layer(w, M)
+        one = call_bytes(base.K, base.N, M, base.rows)
+        R = max(1, math.ceil((3 * L2_BYTES + 1) / (4 * base.N * base.rows)))
+        layers = [base]
+        for r in range(1, R):
+            L = Layer.__new__(Layer)
+            L.__dict__.update(base.__dict__)
+            L.qw = base.qw.clone()
+            L.scales = base.scales.clone()
+            L.ws = q.workspace(M, base.K, base.N)
+            layers.append(L)
+        fn = lambda i: layers[i % R].call(q)  # noqa: E731
+        n = 400 if M <= 64 else 100
+        for g in run_steps(fn, 10, 10):
+            g.replay()
+        secs, _, _ = time_graphs(run_steps(fn, n, 50), ws)
+        secs = max_over_ranks(secs, ws)
+        us = secs / n * 1e6
+        out[str(M)] = {"path": q.qgemm_path_for(M, base.K, base.N), "us": round(us, 2),
+                       "gbs": round(one / us / 1e3, 1),
+                       "tflops": round(2.0 * M * base.K * base.N / us / 1e6, 2)}
+        del layers, base
+        torch.cuda.empty_cache()
+    return out
+
+
+def bench_stack(q, w, steps, ws):
+    """The 80-layer linear stack at M = 1: tokens/s = 1 / (time of all calls)."""
+    calls = []
+    for layer in range(w.layers):
+        for mi in range(len(w.matrices)):
+            calls.append(Layer(w, 1, layer=layer, matrix=mi))
+    total_bytes = sum(call_bytes(c.K, c.N, 1, c.rows) for c in calls)
+    fn = lambda i: calls[i % len(calls)].call(q)  # noqa: E731
+    n = len(calls) * steps
+    for g in run_steps(fn, len(calls), len(calls)):
+        g.replay()
+    secs, _, _ = time_graphs(run_steps(fn, n, len(calls)), ws)
+    secs = max_over_ranks(secs, ws)
+    tok_s = steps / secs
+    out = {"tokens_per_s": round(tok_s, 2), "calls_per_token": len(calls),
+           "bytes_per_token": total_bytes, "gbs": round(total_bytes * tok_s / 1e9, 1)}
+    del calls
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_e2e(q, L, steps, warmup, ws):
     """Public call with host buffers: x in from pinned memory, y back, every step."""
     xh = L.x.cpu().pin_memory()
@@ -356,12 +439,17 @@ def run_ours(args):
     time.sleep(0.2)
     res = bench_decode(q, w, M, args.steps, args.warmup, ws)
     clocks = sampler.summary(res["t0"], res["t1"])
+    wp = W.WORKLOADS[PREFILL]
+    pre = bench_prefill(q, wp, PREFILL_M, max(16, min(160, args.steps // 100)), 5, ws)
+    pre_clocks = sampler.summary(pre["t0"], pre["t1"])
     extra = {}
     if args.full:
-        extra["sweep_gbs"] = {}
+        extra["decode_m_gbs"] = {}
         for m in (2, 4, 8, 16):
             r = bench_decode(q, w, m, min(args.steps, 2000), min(args.warmup, 200), ws)
-            extra["sweep_gbs"][str(m)] = round(r["gbs"], 1)
+            extra["decode_m_gbs"][str(m)] = round(r["gbs"], 1)
+        extra["crossover_sweep"] = bench_sweep(q, W.WORKLOADS[SWEEP], SWEEP_MS, ws)
+        extra["stack"] = bench_stack(q, W.WORKLOADS[STACK], 3, ws)
     e2e = bench_e2e(q, res["layer"], args.steps, args.warmup, ws)
     sampler.stop()
     cpu = cpu_baseline(w, M) if (rank == 0 and ws == 1 and not args.no_cpu) else None
@@ -387,15 +475,31 @@ def run_ours(args):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
                      "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4),
-                     "traffic": traffic_from_profiles("gemv_decode_8192x28672_m1"),
-                     "kernel": "qg::gemv_kernel<1> (+ qg::xprep_kernel, overlapped by PDL; "
+                     "traffic": traffic_from_profiles("gemv_int_decode_8192x28672_m1"),
+                     "kernel": "qg::gemv_int_kernel<1> (+ qg::xprep_int_kernel, overlapped by PDL; "
                                "achieved uses the whole step time)", "peak_source": pk["src"],
                      "bytes_per_launch": res["bytes"]},
+        "prefill": {
+            "workload": PREFILL, "M": PREFILL_M, "K": wp.K, "N": wp.N,
+            "bpw": round(pre["rows"] / (wp.K // 32) + 0.125, 4), "x_dtype": "bf16",
+            "mma_dtype": "f16 (x scaled per row by a power of two, exact)",
+            "value": round(pre["tflops"] * ws, 2), "unit": "TFLOP/s", "ms_per_call": round(pre["ms"], 4),
+            "weight_copies": pre["copies"],
+            "roofline": {"bound": "tensor", "achieved": round(pre["tflops"], 1), "peak": pk["bf16"],
+                         "unit": "TFLOP/s", "frac": round(pre["tflops"] / pk["bf16"], 4),
+                         "peak_sustained": pk["bf16_sust"],
+                         "frac_sustained": round(pre["tflops"] / pk["bf16_sust"], 4),
+                         "traffic": traffic_from_profiles("gemm_prefill_2048x8192x28672"),
+                         "kernel": "qg::gemm_kernel (+ qg::xperm_kernel; achieved uses the whole call)",
+                         "peak_source": pk["src"] + " dense bf16 (fp16 runs at the same rate)"},
+            "clocks": pre_clocks,
+        },
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e["gbs"] * ws, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "steps": e2e["steps"], "how": "eager qgemm() per step; x H2D from pinned, y D2H to pinned"},
         "gpu_launches": 2 * args.steps,
+        "gpu_launches_how": "timed decode region: xprep_int_kernel + gemv_int_kernel per step",
         "clocks": clocks,
     }
     line.update(extra)
@@ -451,6 +555,24 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_target(args):
+    """A few plain calls of one leg, no timing: the command that ncu captures
+    (--profile decode | prefill)."""
+    import mixed_bitwidth_weight_b200 as q
+    torch.cuda.set_device(0)
+    if args.profile == "decode":
+        L = Layer(W.WORKLOADS[HEADLINE], 1)
+    else:
+        L = Layer(W.WORKLOADS[PREFILL], PREFILL_M)
+    for _ in range(args.profile_calls):
+        L.call(q)
+    torch.cuda.synchronize()
+    err = q.qgemm_device_error(clear=True)
+    print(json.dumps({"profile": args.profile, "calls": args.profile_calls, "device_error": err}))
+    if err:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -459,10 +581,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--full", action="store_true", help="also sweep M and the 80-layer stack")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
+                    help="run a few untimed calls of one leg (for ncu) and exit")
+    ap.add_argument("--profile-calls", type=int, default=6)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile:
+        run_profile_target(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -22,11 +22,11 @@
 //
 // Work split as in gemv.cuh: units (256-column tile, 128-row group) split by
 // packed-word cost into one range per CTA (two CTAs per SM for M <= 2, one
-// for M <= 4).  Warp 8 streams each unit into a shared-memory ring of 1 KB
-// rows: its scale row (a bulk copy), its word rows (2D tensor copies of
-// 2^i rows x 256 columns, one per set bit of the row count, so a unit takes
-// two or three copies instead of one per row) and its activation records (a
-// bulk copy).  Weights go out before the wait for the activation kernel;
+// for M <= 4).  Three lanes of warp 8 stream each unit into a shared-memory
+// ring of 1 KB rows: its word rows (2D tensor copies of 2^i rows x 256
+// columns, one per set bit of the row count, so a unit takes two or three
+// copies instead of one per row), its scale row (a bulk copy) and its
+// activation records (a bulk copy).  Weights go out before the wait for the activation kernel;
 // records after it.  Consumer warps 0-7: warp w decodes block w/2 of the unit
 // for the 128 columns of half w%2, four adjacent columns per thread (one
 // 16-byte load per word row); the four block slots are added in shared memory
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
     if (bad) atomicOr(&s_misc[0], 1);
     if (tid == 0) {
         for (int i = 0; i < kGemvSlots; ++i) {
-            mbar_init(&s_full[i], 1);
+            mbar_init(&s_full[i], 3);  // the three issuing lanes of the producer warp
             mbar_init(&s_empty[i], kGemvDecWarps);
         }
         fence_mbar_init();
@@ -350,21 +350,22 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
     };
 
     // =================================================== producer warp
+    // Lanes 0, 1 and 2 split each unit's copies: word rows (2D boxes), the
+    // scale row, the activation records.  One copy instruction takes a fixed
+    // issue time whatever its size, so three issuers keep the ring fuller.
+    // The three lanes take the same ring positions and the same waits, in the
+    // same order, and agree on every wait's outcome, so they issue the same
+    // units.
     if (warp == kGemvDecWarps) {
-        if (lane != 0) return;
+        if (lane > 2) return;
         const uint64_t policy = policy_evict_first();
-        // Copies of unit k = (t, g) at ring row `row`: what & 1 = scale row and
-        // word rows (and the barrier's byte count), what & 2 = activation records.
-        auto issue = [&](int k, int t, int g, int row, int what) {
+        auto issue = [&](int k, int t, int g, int row) {
             const int j0 = g * kGemvGroupBlocks, j1 = min(j0 + kGemvGroupBlocks, nb);
-            const int nblk = j1 - j0;
             const int r0 = s_offs[j0], wrows = s_offs[j1] - r0;
             uint64_t* bar = &s_full[k & (kGemvSlots - 1)];
             uint8_t* dst = s_ring + (size_t)row * kIntRowBytes;
-            if (what & 1) {
-                const int cols = min(kGemvTileCols, p.N - t * kGemvTileCols);
-                mbar_arrive_expect_tx(bar, (uint32_t)(cols * 2 + wrows * kIntRowBytes + nblk * REC));
-                bulk_g2s(dst, p.scales + (size_t)g * p.N + (size_t)t * kGemvTileCols, (uint32_t)cols * 2, bar);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar, (uint32_t)(wrows * kIntRowBytes));
                 int r = 0;
 #pragma unroll 1
                 for (int i = kIntBoxMaps - 1; i >= 0; --i)
@@ -373,13 +374,19 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                                          r0 + r, bar, policy);
                         r += 1 << i;
                     }
+            } else if (lane == 1) {
+                const int cols = min(kGemvTileCols, p.N - t * kGemvTileCols);
+                mbar_arrive_expect_tx(bar, (uint32_t)(cols * 2));
+                bulk_g2s(dst, p.scales + (size_t)g * p.N + (size_t)t * kGemvTileCols, (uint32_t)cols * 2, bar);
+            } else {
+                const int nblk = j1 - j0;
+                mbar_arrive_expect_tx(bar, (uint32_t)(nblk * REC));
+                bulk_g2s(dst + (size_t)(1 + wrows) * kIntRowBytes, p.rec + (size_t)j0 * REC, (uint32_t)nblk * REC,
+                         bar);
             }
-            if (what & 2)
-                bulk_g2s(dst + (size_t)(1 + wrows) * kIntRowBytes, p.rec + (size_t)j0 * REC,
-                         (uint32_t)nblk * REC, bar);
         };
         // Units that fit the ring and the slots before any release: weights
-        // first, then (once the activation kernel is done) their records.
+        // and scales first, then (once the activation kernel is done) records.
         int npre = 0;
         {
             int pp = 0, gg = gf;
@@ -399,15 +406,16 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
         int64_t total = 0;
         int t = t0, g = gf;
         for (int k = 0; k < npre; ++k) {
-            issue(k, t, g, ring_alloc(pos, total, rows_of(g), R), 1);
+            const int row = ring_alloc(pos, total, rows_of(g), R);
+            if (lane != 2) issue(k, t, g, row);
             if (++g == ng) { g = 0; ++t; }
         }
-        asm volatile("griddepcontrol.wait;" ::: "memory");  // activation records come from xprep_int
-        {
+        if (lane == 2) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");  // activation records come from xprep_int
             int pp = 0, tt = t0, gg = gf;
             int64_t tot = 0;
             for (int k = 0; k < npre; ++k) {
-                issue(k, tt, gg, ring_alloc(pp, tot, rows_of(gg), R), 2);
+                issue(k, tt, gg, ring_alloc(pp, tot, rows_of(gg), R));
                 if (++gg == ng) { gg = 0; ++tt; }
             }
         }
@@ -416,13 +424,14 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
         int k_rel = 0, g_rel = gf;
         bool ok = true;
         int k = npre;
-        for (; k < nunits && ok; ++k) {
+        for (; k < nunits; ++k) {
             const int need = rows_of(g);
             int ppos = pos;
             int64_t ptotal = total;
             ring_alloc(ppos, ptotal, need, R);
             while (k - k_rel >= kGemvSlots || ptotal - total_rel > R) {
-                if (!mbar_wait(&s_empty[k_rel & (kGemvSlots - 1)], (uint32_t)((k_rel / kGemvSlots) & 1))) {
+                const bool w = mbar_wait(&s_empty[k_rel & (kGemvSlots - 1)], (uint32_t)((k_rel / kGemvSlots) & 1));
+                if (!__all_sync(0x7u, w)) {
                     ok = false;
                     break;
                 }
@@ -431,7 +440,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                 if (++g_rel == ng) g_rel = 0;
             }
             if (!ok) break;
-            issue(k, t, g, ring_alloc(pos, total, need, R), 3);
+            issue(k, t, g, ring_alloc(pos, total, need, R));
             if (++g == ng) { g = 0; ++t; }
         }
         if (!ok) {
