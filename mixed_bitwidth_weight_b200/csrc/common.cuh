@@ -124,6 +124,16 @@ QG_DEV void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* 
 }
 
 // 2D tensor copy global -> this CTA's shared memory of the box at (x, y) of
+// the tensor map, completing on an mbarrier (same rules as below).
+QG_DEV void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 2D tensor copy global -> this CTA's shared memory of the box at (x, y) of
 // the tensor map (x in elements, a multiple of 16 bytes; y in rows), with an
 // L2 cache policy.  dst 128-byte aligned.  The whole box counts toward the
 // mbarrier's transaction bytes, out-of-range elements arriving as zeros.

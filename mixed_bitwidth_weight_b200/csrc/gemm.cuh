@@ -127,14 +127,6 @@ __global__ void __launch_bounds__(256) xperm_kernel(const XpermParams p) {
     }
 }
 
-QG_DEV void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // Two fp32 values -> one 32-bit pair of the activation type, RNE; lo in the
 // low half.
 template <bool BF16>

@@ -358,7 +358,6 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
     // units.
     if (warp == kGemvDecWarps) {
         if (lane > 2) return;
-        const uint64_t policy = policy_evict_first();
         auto issue = [&](int k, int t, int g, int row) {
             const int j0 = g * kGemvGroupBlocks, j1 = min(j0 + kGemvGroupBlocks, nb);
             const int r0 = s_offs[j0], wrows = s_offs[j1] - r0;
@@ -370,8 +369,8 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
 #pragma unroll 1
                 for (int i = kIntBoxMaps - 1; i >= 0; --i)
                     if (wrows & (1 << i)) {
-                        tma_load_2d_hint(dst + (size_t)(1 + r) * kIntRowBytes, &maps.box[i], t * kGemvTileCols,
-                                         r0 + r, bar, policy);
+                        tma_load_2d(dst + (size_t)(1 + r) * kIntRowBytes, &maps.box[i], t * kGemvTileCols, r0 + r,
+                                    bar);
                         r += 1 << i;
                     }
             } else if (lane == 1) {
