@@ -115,7 +115,8 @@ int qgemm_path_for(int M, int K, int N);
 
 /* Launch plan qgemm() would use for this shape on the current device (or on a
  * 148-SM device when no GPU is visible).  out[0] = kernel family (as
- * qgemm_path_for), out[1] = grid size, out[2] = shared-memory ring rows (GEMV),
+ * qgemm_path_for), out[1] = grid size, out[2] = shared-memory ring rows (GEMV)
+ * or number of k splits (GEMM),
  * out[3] = CTAs resident per SM, out[4] = dynamic shared
  * memory bytes, out[5] = SM count used.  Host only; returns a qgemm_status. */
 int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out);

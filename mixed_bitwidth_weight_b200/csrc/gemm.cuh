@@ -60,7 +60,9 @@ struct GemmParams {
     const int32_t* offs;
     int64_t qw_rows;
     __half* y;
-    int M, K, N, nb, mtiles, x_bf16;
+    int* tickets;      // [tiles] (split K only)
+    float* partial;    // [tiles][ksplit][256][256] fp32 partial sums (split K only)
+    int M, K, N, nb, mtiles, ntiles, ksplit, x_bf16;
 };
 
 struct XpermParams {
@@ -204,9 +206,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int* s_misc = reinterpret_cast<int*>(acc_full + 1);  // [0] bad schedule, [1] abort, [2] tmem base
     int32_t* s_offs = s_misc + 8;
 
-    const int mt = blockIdx.x % p.mtiles, ntile = blockIdx.x / p.mtiles;
+    // blockIdx.x = (ks * ntiles + ntile) * mtiles + mt: CTAs next to each
+    // other share the weight tile and k range
+    const int mt = blockIdx.x % p.mtiles;
+    const int ntile = (blockIdx.x / p.mtiles) % p.ntiles;
+    const int ks = blockIdx.x / (p.mtiles * p.ntiles);
+    const int tile = ntile * p.mtiles + mt;
     const int m0 = mt * kGemmBM, n0 = ntile * kGemmBN;
-    const int nk = (p.K + kGemmBK - 1) / kGemmBK;
+    const int nk_all = (p.K + kGemmBK - 1) / kGemmBK;
+    const int kb = (int)((int64_t)ks * nk_all / p.ksplit);
+    const int nk = (int)((int64_t)(ks + 1) * nk_all / p.ksplit) - kb;  // this CTA's k steps
+    const bool two = m0 + 128 < p.M;  // second 128-row half holds rows of x
 
     // ---- schedule into shared memory, validated before any weight access
     if (tid < 8) s_misc[tid] = 0;
@@ -260,11 +270,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ok = false;
                     break;
                 }
+                const int gi = kb + i;  // global k step
                 mbar_arrive_expect_tx(&a_full[sa], (uint32_t)kGemmABytes);
-                tma_load_2d(sA + sa * kGemmABytes, &maps.a, i * kGemmBK, m0, &a_full[sa]);
-                const int j0 = 2 * i, j1 = min(j0 + 2, nb);
+                tma_load_2d(sA + sa * kGemmABytes, &maps.a, gi * kGemmBK, m0, &a_full[sa]);
+                const int j0 = 2 * gi, j1 = min(j0 + 2, nb);
                 const int r0 = s_offs[j0], rows = s_offs[j1] - r0;
-                const int g = (i * kGemmBK) / 128;
+                const int g = (gi * kGemmBK) / 128;
                 const int cols = min(kGemmBN, p.N - n0);
                 uint8_t* dst = sR + sr * kGemmRBytes;
                 mbar_arrive_expect_tx(&r_full[sr], (uint32_t)(cols * 2 + rows * 1024));
@@ -302,6 +313,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+                        if (h == 1 && !two) continue;
                         const uint64_t ad = smem_desc(a_addr + h * (128 * 128) + kk * 32, 16, 1024, 2);
                         const uint64_t bd = smem_desc(b_addr + kk * 32, 16, 1024, 2);
                         tc_mma_ss(tmem + h * kGemmBN, ad, bd, kIdesc, (i | kk) != 0);
@@ -324,7 +336,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint8_t* raw = sR + sr * kGemmRBytes;
             const float s = __half2float(reinterpret_cast<const __half*>(raw)[n]);
             uint8_t* brow = sB + sb * kGemmBBytes + n * 128;
-            const int j0 = 2 * i;
+            const int j0 = 2 * (kb + i);
             const int r0 = s_offs[j0];
 #pragma unroll
             for (int blk = 0; blk < 2; ++blk) {
@@ -351,30 +363,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 mbar_arrive(&r_empty[sr]);
             }
         }
-        // ---- epilogue: TMEM -> y (fp16)
+        // ---- epilogue: TMEM -> y (fp16), or fp32 partial sums under split K
         const bool ok = mbar_wait(acc_full, 0) && !s_misc[1];
         tc_fence_after();
-        if (ok) {
-            const int q = warp & 3, h = (warp - 2) >> 2;
-            const int row = m0 + h * 128 + q * 32 + lane;
+        const int q = warp & 3, h = (warp - 2) >> 2;
+        const int rl = h * 128 + q * 32 + lane;  // row within the tile
+        const int row = m0 + rl;
+        const int sh = (p.x_bf16 && row < p.M) ? p.xshift[row] : 0;
+        const float g1 = __int_as_float((127 + sh / 2) << 23), g2 = __int_as_float((127 + (sh - sh / 2)) << 23);
+        auto store_y = [&](int r, int c, const float (&v)[16], float s1, float s2) {
+            uint32_t hv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const __half2 t = __floats2half2_rn(v[2 * u] * s1 * s2, v[2 * u + 1] * s1 * s2);
+                hv[u] = *reinterpret_cast<const uint32_t*>(&t);
+            }
+            __half* dst = p.y + (size_t)r * p.N + n0 + c;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            if (n0 + c + 8 < p.N) *reinterpret_cast<uint4*>(dst + 8) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        };
+        if (ok && (h == 0 || two)) {
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + h * kGemmBN;
-            const int sh = (p.x_bf16 && row < p.M) ? p.xshift[row] : 0;
-            const float g1 = __int_as_float((127 + sh / 2) << 23), g2 = __int_as_float((127 + (sh - sh / 2)) << 23);
+            float* part = p.partial + ((size_t)tile * p.ksplit + ks) * (kGemmBM * kGemmBN) + (size_t)rl * kGemmBN;
 #pragma unroll 1
             for (int c = 0; c < kGemmBN; c += 16) {
                 float v[16];
                 tmem_ld16(taddr + c, v);
-                if (row < p.M && n0 + c < p.N) {
-                    uint32_t hv[8];
+                if (p.ksplit == 1) {
+                    if (row < p.M && n0 + c < p.N) store_y(row, c, v, g1, g2);
+                } else {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const __half2 t = __floats2half2_rn(v[2 * u] * g1 * g2, v[2 * u + 1] * g1 * g2);
-                        hv[u] = *reinterpret_cast<const uint32_t*>(&t);
-                    }
-                    __half* dst = p.y + (size_t)row * p.N + n0 + c;
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                    if (n0 + c + 8 < p.N) *reinterpret_cast<uint4*>(dst + 8) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+                    for (int u = 0; u < 4; ++u)
+                        *reinterpret_cast<float4*>(part + c + 4 * u) =
+                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
                 }
+            }
+        }
+        if (p.ksplit > 1) {
+            // the last of the tile's ksplit CTAs adds the partial sums
+            __threadfence();
+            named_bar_sync(1, kGemmDecWarps * 32);
+            if (tid == 64) s_misc[3] = (ok && !s_misc[1]) ? (atomicAdd(&p.tickets[tile], 1) == p.ksplit - 1) : 0;
+            named_bar_sync(1, kGemmDecWarps * 32);
+            if (s_misc[3]) {
+                __threadfence();
+                const int r2 = tid - 64;  // one tile row per thread
+                const int row2 = m0 + r2;
+                if (row2 < p.M) {
+                    const int sh2 = p.x_bf16 ? p.xshift[row2] : 0;
+                    const float s1 = __int_as_float((127 + sh2 / 2) << 23);
+                    const float s2 = __int_as_float((127 + (sh2 - sh2 / 2)) << 23);
+                    const float* base_p = p.partial + (size_t)tile * p.ksplit * (kGemmBM * kGemmBN) + (size_t)r2 * kGemmBN;
+#pragma unroll 1
+                    for (int c = 0; c < kGemmBN && n0 + c < p.N; c += 16) {
+                        float v[16];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) v[u] = 0.f;
+                        for (int kq = 0; kq < p.ksplit; ++kq) {
+                            const float* src = base_p + (size_t)kq * (kGemmBM * kGemmBN) + c;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const float4 f = __ldcg(reinterpret_cast<const float4*>(src) + u);
+                                v[4 * u] += f.x;
+                                v[4 * u + 1] += f.y;
+                                v[4 * u + 2] += f.z;
+                                v[4 * u + 3] += f.w;
+                            }
+                        }
+                        store_y(row2, c, v, s1, s2);
+                    }
+                }
+                if (tid == 64) p.tickets[tile] = 0;
             }
         }
     }

@@ -369,9 +369,30 @@ int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t
 // ------------------------------------------------------------------ GEMM
 int gemm_mtiles(int M) { return (M + kGemmBM - 1) / kGemmBM; }
 int gemm_ntiles(int N) { return (N + kGemmBN - 1) / kGemmBN; }
-// Workspace: [x_p fp16 M x K][row shifts int32 M].
-size_t gemm_ws_xshift(int M, int K) { return align_up((size_t)M * K * 2, 256); }
-size_t gemm_ws_bytes(int M, int K) { return gemm_ws_xshift(M, K) + align_up((size_t)M * 4, 256); }
+// Split K when the output tiles cannot fill the GPU: as many splits as keep
+// one wave (tiles * ksplit <= SMs), each split at least 8 k steps long.
+int gemm_ksplit(int M, int K, int N, int sms) {
+    const int64_t tiles = (int64_t)gemm_mtiles(M) * gemm_ntiles(N);
+    if (tiles >= sms) return 1;
+    const int nk = (K + kGemmBK - 1) / kGemmBK;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(sms / tiles, nk / 8));
+}
+
+// Workspace: [x_p fp16 M x K][row shifts int32 M][tickets][fp32 partial tiles].
+struct GemmWs {
+    size_t xshift, tickets, partial, total;
+};
+
+GemmWs gemm_ws_layout(int M, int K, int N, int sms) {
+    const int64_t tiles = (int64_t)gemm_mtiles(M) * gemm_ntiles(N);
+    const int ks = gemm_ksplit(M, K, N, sms);
+    GemmWs w;
+    w.xshift = align_up((size_t)M * K * 2, 256);
+    w.tickets = w.xshift + align_up((size_t)M * 4, 256);
+    w.partial = w.tickets + align_up((size_t)tiles * 4, 256);
+    w.total = w.partial + (ks > 1 ? (size_t)tiles * ks * kGemmBM * kGemmBN * 4 : 0);
+    return w;
+}
 size_t gemm_smem(int nb) { return (size_t)kGemmFixedSmem + 512 + (size_t)(nb + 1) * 4; }
 
 int make_gemm_maps(const void* xp, int x_dtype, int M, int K, const uint32_t* qw, int64_t qw_rows, int N,
@@ -405,7 +426,8 @@ int make_gemm_maps(const void* xp, int x_dtype, int M, int K, const uint32_t* qw
 int run_gemm(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
              const uint16_t* scales, const uint8_t* bits, const int32_t* offs, int M, int K, int N, uint16_t* y,
              void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev) {
-    if (ws == nullptr || ws_bytes < gemm_ws_bytes(M, K)) return QGEMM_ERR_WORKSPACE;
+    const GemmWs L = gemm_ws_layout(M, K, N, dev->sms);
+    if (ws == nullptr || ws_bytes < L.total) return QGEMM_ERR_WORKSPACE;
     const int nb = K / kBlockRows;
     const size_t smem = gemm_smem(nb);
     if (smem > (size_t)227 * 1024) return QGEMM_ERR_UNSUPPORTED;
@@ -416,7 +438,7 @@ int run_gemm(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
             return QGEMM_ERR_CUDA;
         dev->gemm_attr[0] = true;
     }
-    int* xshift = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + gemm_ws_xshift(M, K));
+    int* xshift = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.xshift);
     GemmMaps maps;
     int st = make_gemm_maps(ws, x_dtype, M, K, qw, qw_rows, N, &maps);
     if (st != QGEMM_OK) return st;
@@ -444,8 +466,12 @@ int run_gemm(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     p.N = N;
     p.nb = nb;
     p.mtiles = gemm_mtiles(M);
+    p.ntiles = gemm_ntiles(N);
+    p.ksplit = gemm_ksplit(M, K, N, dev->sms);
+    p.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.tickets);
+    p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.partial);
     p.x_bf16 = bf16;
-    const unsigned grid = (unsigned)((int64_t)gemm_mtiles(M) * gemm_ntiles(N));
+    const unsigned grid = (unsigned)((int64_t)p.mtiles * p.ntiles * p.ksplit);
     gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(p, maps);
     return launch_status();
 }
@@ -559,7 +585,7 @@ size_t qgemm_workspace_bytes(int M, int K, int N) {
     const int path = qgemm_path_for(M, K, N);
     if (path == kPathGemvInt) return int_ws_layout(M, K, N, sms).total;
     if (path == kPathGemvTc) return gemv_ws_layout(M, K, N, sms).total;
-    return gemm_ws_bytes(M, K);
+    return gemm_ws_layout(M, K, N, sms).total;
 }
 
 int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out) {
@@ -593,8 +619,8 @@ int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out) {
         return QGEMM_OK;
     }
     if (out[0] == kPathGemm) {
-        out[1] = (int64_t)gemm_mtiles(M) * gemm_ntiles(N);
-        out[2] = 0;
+        out[1] = (int64_t)gemm_mtiles(M) * gemm_ntiles(N) * gemm_ksplit(M, K, N, sms);
+        out[2] = gemm_ksplit(M, K, N, sms);
         out[3] = 1;
         out[4] = (int64_t)gemm_smem(K / kBlockRows);
         return QGEMM_OK;

@@ -133,4 +133,8 @@ def test_gemm_plan_and_workspace():
     assert plan["smem"] <= 227 * 1024
     assert q.qgemm_workspace_bytes(2048, 8192, 28672) >= 2048 * 8192 * 2
     big = q.qgemm_plan_info(17, 65536, 8, 2 * 2048)
-    assert big["smem"] <= 227 * 1024 and big["grid"] == 1
+    assert big["smem"] <= 227 * 1024
+    # one output tile: k is split so that the SMs have work, 8+ k steps each
+    ks = big["ring"]
+    assert 1 < ks <= 148 and big["grid"] == ks and (65536 // 64) // ks >= 8
+    assert q.qgemm_workspace_bytes(17, 65536, 8) >= 17 * 65536 * 2 + ks * 256 * 256 * 4

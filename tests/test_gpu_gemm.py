@@ -49,6 +49,18 @@ def test_gemm_parity(q, M, K, N, x_dtype):
     P.check_close(run(q, pr), P.ref_y(pr))
 
 
+@pytest.mark.parametrize("M,K,N", [(64, 8192, 512), (200, 4096, 256), (33, 2048, 1032)])
+def test_gemm_split_k(q, M, K, N):
+    """Few output tiles: k is split across CTAs and the last one adds the
+    partial sums (deterministic, workspace tickets back to zero)."""
+    plan = q.qgemm_plan_info(M, K, N, int(P.make(K, 8, kind="shuffled", seed=1)["offs"][-1]))
+    assert plan["ring"] > 1                       # k splits
+    pr = P.make(K, N, M=M, kind="shuffled", seed=M + N, x_dtype=torch.bfloat16)
+    a = run(q, pr)
+    P.check_close(a, P.ref_y(pr))
+    assert torch.equal(a, run(q, pr))
+
+
 @pytest.mark.parametrize("kind", ["u2", "u3", "u4", "u5", "u6", "u8", "sorted"])
 def test_gemm_parity_every_width(q, kind):
     pr = P.make(512, 520, M=96, kind=kind, seed=5)
