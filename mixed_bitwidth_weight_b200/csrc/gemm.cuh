@@ -16,9 +16,10 @@
 //                  tcgen05.mma kind::f16, M = 128, N = 256, K = 16, both
 //                  operands from shared memory;
 //     warps 2-9  - dequantise: thread n decodes the 64 codes of column n in
-//                  the step (two 32-row blocks, each at its own width), forms
-//                  w = (q - 2^(b-1)) * s exactly in fp32, rounds once to fp16
-//                  (the bit-exact dequantised weight) and writes row n of the B tile in the
+//                  the step (two 32-row blocks, each at its own width) two
+//                  per instruction in fp16 pairs, forms w = (q - 2^(b-1)) * s
+//                  with one rounding (the bit-exact dequantised weight) and
+//                  writes row n of the B tile in the
 //                  K-major 128-byte-swizzled layout the MMA reads; after the
 //                  last step they move the accumulators TMEM -> fp16 y.
 // Every wait is bounded; a timeout sets the device error word, the CTA skips
@@ -68,12 +69,28 @@ struct GemmParams {
 struct XpermParams {
     const uint16_t* x;
     const int32_t* perm;
+    const uint8_t* bits;
     uint16_t* xp;
     int* xshift;   // [M] per-row power-of-two shift (bf16 input)
     int M, K, x_bf16;
 };
 
-// x_p[m][k] = fp16(x[m][perm[k]] * 2^-shift[m]), one CTA per row, 8 k per
+// Order of the k positions of one 32-row block inside the B tile (and so in
+// x_p): the dequantiser extracts two codes per 32-bit word into the two fp16
+// halves with one shift and one mask, so position pair i holds codes that sit
+// 16 bits apart.  b = 2: pair (8w+s) = codes (16w+s, 16w+s+8); b = 4: pair
+// (4w+s) = codes (8w+s, 8w+s+4); b = 8: pair (2w+s) = codes (4w+s, 4w+s+2);
+// 3, 5, 6: natural order.
+QG_DEV int gemm_code_of_k(int b, int k) {
+    const int i = k >> 1, h = k & 1;
+    if (b == 2) return 16 * (i >> 3) + (i & 7) + 8 * h;
+    if (b == 4) return 8 * (i >> 2) + (i & 3) + 4 * h;
+    if (b == 8) return 4 * (i >> 1) + (i & 1) + 2 * h;
+    return k;
+}
+
+// x_p[m][k] = fp16(x[m][perm[k']] * 2^-shift[m]), k' = the code the B tile
+// holds at position k (gemm_code_of_k), one CTA per row, 8 k per
 // thread step (16-byte stores).  fp16 input: shift 0, a plain gather.  bf16
 // input: shift puts the row's largest magnitude in [2^14, 2^15), so the
 // conversion to fp16 is exact for every value within 2^24 of the maximum;
@@ -103,9 +120,11 @@ __global__ void __launch_bounds__(256) xperm_kernel(const XpermParams p) {
     const int s1 = shift / 2, s2 = shift - shift / 2;  // 2^-shift as two normal factors
     const float f1 = __int_as_float((127 - s1) << 23), f2 = __int_as_float((127 - s2) << 23);
     for (int k0 = threadIdx.x * 8; k0 < p.K; k0 += blockDim.x * 8) {
-        const int4 i0 = *reinterpret_cast<const int4*>(p.perm + k0);
-        const int4 i1 = *reinterpret_cast<const int4*>(p.perm + k0 + 4);
-        const int idx[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+        const int blk = k0 >> 5;
+        const int b = p.bits[blk];  // the GEMM refuses a schedule with a bad width
+        int idx[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) idx[u] = p.perm[blk * 32 + gemm_code_of_k(b, (k0 & 31) + u)];
         uint32_t v[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -129,51 +148,61 @@ __global__ void __launch_bounds__(256) xperm_kernel(const XpermParams p) {
     }
 }
 
-// Two fp32 values -> one 32-bit pair of the activation type, RNE; lo in the
-// low half.
-template <bool BF16>
-QG_DEV uint32_t pack2(float lo, float hi) {
+QG_DEV uint32_t h2sub(uint32_t a, uint32_t b) {
     uint32_t d;
-    if constexpr (BF16) asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    else asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+QG_DEV uint32_t h2mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
-// The 32 codes of one block for this thread's column, dequantised:
-// out[i] = pair (w[2i], w[2i+1]).  w0 = word row 0 of the block at this column,
-// word rows 1 KB apart.  (2^23 + q) - (2^23 + z) = q - z exactly, and (q - z) * s
-// has at most 19 significant bits, so the one rounding is the cvt.
-template <int B, bool BF16>
-QG_DEV void dequant_block32(const uint8_t* w0, float s, uint32_t (&out)[16]) {
+// The 32 codes of one block for this thread's column, dequantised to fp16
+// pairs in the B tile's order (gemm_code_of_k).  Two codes at bits p and
+// p + 16 of a word become (1024 + q) in each half with one mask and an OR of
+// 0x6400 (the fp16 of 1024); subtracting 1024 + z is exact and the multiply
+// by the fp16 scale is the one rounding: bit-exact with qgemm_dequant.
+// w0 = word row 0 of the block at this column, word rows 1 KB apart.
+template <int B>
+QG_DEV void dequant_block32(const uint8_t* w0, uint32_t s2, uint32_t (&out)[16]) {
     constexpr uint32_t mask = (1u << B) - 1u;
-    const float zoff = 8388608.f + (float)(1 << (B - 1));
+    const uint32_t zoff = 0x64006400u + (((uint32_t)1 << (B - 1)) * 0x00010001u);  // 1024 + z in both halves
     uint32_t w[B];
 #pragma unroll
     for (int i = 0; i < B; ++i) w[i] = *reinterpret_cast<const uint32_t*>(w0 + i * 1024);
+    if constexpr (B == 2 || B == 4 || B == 8) {
+        constexpr int per = 16 / B;  // pairs per word
 #pragma unroll
-    for (int r = 0; r < 32; r += 2) {
-        float f[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int bit = (r + u) * B, wi = bit >> 5, sh = bit & 31;
-            uint32_t q;
-            if (sh + B <= 32) q = (w[wi] >> sh) & mask;
-            else q = __funnelshift_r(w[wi], w[wi + 1 < B ? wi + 1 : wi], sh) & mask;
-            f[u] = (__uint_as_float(0x4B000000u | q) - zoff) * s;
+        for (int i = 0; i < 16; ++i) {
+            const int wi = i / per, sft = (i % per) * B;
+            const uint32_t h = lop3_and_or(w[wi] >> sft, mask * 0x00010001u, 0x64006400u);
+            out[i] = h2mul(h2sub(h, zoff), s2);
         }
-        out[r / 2] = pack2<BF16>(f[0], f[1]);
+    } else {  // 3, 5, 6: codes 2i and 2i+1 in natural order
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            uint32_t q[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int bit = (2 * i + u) * B, wi = bit >> 5, sh = bit & 31;
+                if (sh + B <= 32) q[u] = (w[wi] >> sh) & mask;
+                else q[u] = __funnelshift_r(w[wi], w[wi + 1 < B ? wi + 1 : wi], sh) & mask;
+            }
+            out[i] = h2mul(h2sub((q[0] | (q[1] << 16)) | 0x64006400u, zoff), s2);
+        }
     }
 }
 
-template <bool BF16>
-QG_DEV void dequant_block32_any(int b, const uint8_t* w0, float s, uint32_t (&out)[16]) {
+QG_DEV void dequant_block32_any(int b, const uint8_t* w0, uint32_t s2, uint32_t (&out)[16]) {
     switch (b) {
-        case 2: dequant_block32<2, BF16>(w0, s, out); break;
-        case 3: dequant_block32<3, BF16>(w0, s, out); break;
-        case 4: dequant_block32<4, BF16>(w0, s, out); break;
-        case 5: dequant_block32<5, BF16>(w0, s, out); break;
-        case 6: dequant_block32<6, BF16>(w0, s, out); break;
-        default: dequant_block32<8, BF16>(w0, s, out); break;
+        case 2: dequant_block32<2>(w0, s2, out); break;
+        case 3: dequant_block32<3>(w0, s2, out); break;
+        case 4: dequant_block32<4>(w0, s2, out); break;
+        case 5: dequant_block32<5>(w0, s2, out); break;
+        case 6: dequant_block32<6>(w0, s2, out); break;
+        default: dequant_block32<8>(w0, s2, out); break;
     }
 }
 
@@ -334,7 +363,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 break;
             }
             const uint8_t* raw = sR + sr * kGemmRBytes;
-            const float s = __half2float(reinterpret_cast<const __half*>(raw)[n]);
+            const uint32_t sbits = reinterpret_cast<const uint16_t*>(raw)[n];
+            const uint32_t s2 = sbits | (sbits << 16);
             uint8_t* brow = sB + sb * kGemmBBytes + n * 128;
             const int j0 = 2 * (kb + i);
             const int r0 = s_offs[j0];
@@ -343,8 +373,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int j = j0 + blk;
                 uint32_t out[16];
                 if (j < nb) {
-                    dequant_block32_any<BF16>(s_offs[j + 1] - s_offs[j],
-                                              raw + 1024 + (size_t)(s_offs[j] - r0) * 1024 + n * 4, s, out);
+                    dequant_block32_any(s_offs[j + 1] - s_offs[j],
+                                        raw + 1024 + (size_t)(s_offs[j] - r0) * 1024 + n * 4, s2, out);
                 } else {
 #pragma unroll
                     for (int u = 0; u < 16; ++u) out[u] = 0;

@@ -446,6 +446,7 @@ int run_gemm(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     XpermParams xq;
     xq.x = static_cast<const uint16_t*>(x);
     xq.perm = perm;
+    xq.bits = bits;
     xq.xp = static_cast<uint16_t*>(ws);
     xq.xshift = xshift;
     xq.M = M;
