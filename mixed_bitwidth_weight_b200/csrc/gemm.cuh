@@ -61,9 +61,11 @@ struct GemmParams {
     const int32_t* offs;
     int64_t qw_rows;
     __half* y;
-    int* tickets;      // [tiles] (split K only)
-    float* partial;    // [tiles][ksplit][256][256] fp32 partial sums (split K only)
-    int M, K, N, nb, mtiles, ntiles, ksplit, x_bf16;
+    int* tickets;      // [tiles] (split tiles only)
+    float* partial;    // [split tiles][256][256] fp32 sums, zero between calls
+    int M, K, N, nb, mtiles, ntiles, x_bf16;
+    int full_tiles;    // tiles done whole, one per CTA (whole waves of the grid)
+    int ksplit;        // k splits of each remaining tile (the last wave)
 };
 
 struct XpermParams {
@@ -235,16 +237,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int* s_misc = reinterpret_cast<int*>(acc_full + 1);  // [0] bad schedule, [1] abort, [2] tmem base
     int32_t* s_offs = s_misc + 8;
 
-    // blockIdx.x = (ks * ntiles + ntile) * mtiles + mt: CTAs next to each
-    // other share the weight tile and k range
-    const int mt = blockIdx.x % p.mtiles;
-    const int ntile = (blockIdx.x / p.mtiles) % p.ntiles;
-    const int ks = blockIdx.x / (p.mtiles * p.ntiles);
-    const int tile = ntile * p.mtiles + mt;
+    // CTAs below full_tiles take one whole tile each (tile = ntile * mtiles +
+    // mt, so neighbours share the weight tile); the rest split the k range of
+    // the remaining tiles ksplit ways (neighbours: same k range)
+    const int full = p.full_tiles;
+    const bool split = (int)blockIdx.x >= full;
+    const int rest = p.mtiles * p.ntiles - full;
+    const int ks = split ? (int)(blockIdx.x - full) / rest : 0;
+    const int tile = split ? full + (int)(blockIdx.x - full) % rest : (int)blockIdx.x;
+    const int nsplit = split ? p.ksplit : 1;
+    const int mt = tile % p.mtiles, ntile = tile / p.mtiles;
     const int m0 = mt * kGemmBM, n0 = ntile * kGemmBN;
     const int nk_all = (p.K + kGemmBK - 1) / kGemmBK;
-    const int kb = (int)((int64_t)ks * nk_all / p.ksplit);
-    const int nk = (int)((int64_t)(ks + 1) * nk_all / p.ksplit) - kb;  // this CTA's k steps
+    const int kb = (int)((int64_t)ks * nk_all / nsplit);
+    const int nk = (int)((int64_t)(ks + 1) * nk_all / nsplit) - kb;  // this CTA's k steps
     const bool two = m0 + 128 < p.M;  // second 128-row half holds rows of x
 
     // ---- schedule into shared memory, validated before any weight access
@@ -414,54 +420,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         };
         if (ok && (h == 0 || two)) {
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + h * kGemmBN;
-            float* part = p.partial + ((size_t)tile * p.ksplit + ks) * (kGemmBM * kGemmBN) + (size_t)rl * kGemmBN;
+            float* acc = p.partial + (size_t)(tile - full) * (kGemmBM * kGemmBN) + (size_t)rl * kGemmBN;
 #pragma unroll 1
             for (int c = 0; c < kGemmBN; c += 16) {
                 float v[16];
                 tmem_ld16(taddr + c, v);
-                if (p.ksplit == 1) {
+                if (nsplit == 1) {
                     if (row < p.M && n0 + c < p.N) store_y(row, c, v, g1, g2);
-                } else {
+                } else if (row < p.M) {
+                    // fire-and-forget vector reductions into the tile's fp32 sum
+                    // (only columns of y: the accumulator outside stays zero)
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        *reinterpret_cast<float4*>(part + c + 4 * u) =
-                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                        if (n0 + c + 4 * u < p.N)
+                            atomicAdd(reinterpret_cast<float4*>(acc + c + 4 * u),
+                                      make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]));
                 }
             }
         }
-        if (p.ksplit > 1) {
-            // the last of the tile's ksplit CTAs adds the partial sums
+        if (nsplit > 1) {
+            // the last of the tile's nsplit CTAs converts the sum to y and
+            // leaves the accumulator at zero for the next call
             __threadfence();
             named_bar_sync(1, kGemmDecWarps * 32);
-            if (tid == 64) s_misc[3] = (ok && !s_misc[1]) ? (atomicAdd(&p.tickets[tile], 1) == p.ksplit - 1) : 0;
+            if (tid == 64) s_misc[3] = (ok && !s_misc[1]) ? (atomicAdd(&p.tickets[tile], 1) == nsplit - 1) : 0;
             named_bar_sync(1, kGemmDecWarps * 32);
             if (s_misc[3]) {
                 __threadfence();
-                const int r2 = tid - 64;  // one tile row per thread
-                const int row2 = m0 + r2;
-                if (row2 < p.M) {
+                float4* acc4 = reinterpret_cast<float4*>(p.partial + (size_t)(tile - full) * (kGemmBM * kGemmBN));
+                const int t = tid - 64;
+#pragma unroll 4
+                for (int f = t; f < kGemmBM * kGemmBN / 4; f += kGemmDecWarps * 32) {
+                    const int r2 = f / (kGemmBN / 4), c4 = (f % (kGemmBN / 4)) * 4;
+                    const int row2 = m0 + r2;
+                    if (row2 >= p.M || n0 + c4 >= p.N) continue;
+                    const float4 a = __ldcg(acc4 + f);
+                    __stcg(acc4 + f, make_float4(0.f, 0.f, 0.f, 0.f));
                     const int sh2 = p.x_bf16 ? p.xshift[row2] : 0;
                     const float s1 = __int_as_float((127 + sh2 / 2) << 23);
                     const float s2 = __int_as_float((127 + (sh2 - sh2 / 2)) << 23);
-                    const float* base_p = p.partial + (size_t)tile * p.ksplit * (kGemmBM * kGemmBN) + (size_t)r2 * kGemmBN;
-#pragma unroll 1
-                    for (int c = 0; c < kGemmBN && n0 + c < p.N; c += 16) {
-                        float v[16];
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) v[u] = 0.f;
-                        for (int kq = 0; kq < p.ksplit; ++kq) {
-                            const float* src = base_p + (size_t)kq * (kGemmBM * kGemmBN) + c;
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const float4 f = __ldcg(reinterpret_cast<const float4*>(src) + u);
-                                v[4 * u] += f.x;
-                                v[4 * u + 1] += f.y;
-                                v[4 * u + 2] += f.z;
-                                v[4 * u + 3] += f.w;
-                            }
-                        }
-                        store_y(row2, c, v, s1, s2);
-                    }
+                    const __half2 lo = __floats2half2_rn(a.x * s1 * s2, a.y * s1 * s2);
+                    const __half2 hi = __floats2half2_rn(a.z * s1 * s2, a.w * s1 * s2);
+                    *reinterpret_cast<uint2*>(p.y + (size_t)row2 * p.N + n0 + c4) =
+                        make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
                 }
                 if (tid == 64) p.tickets[tile] = 0;
             }

@@ -369,13 +369,29 @@ int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t
 // ------------------------------------------------------------------ GEMM
 int gemm_mtiles(int M) { return (M + kGemmBM - 1) / kGemmBM; }
 int gemm_ntiles(int N) { return (N + kGemmBN - 1) / kGemmBN; }
-// Split K when the output tiles cannot fill the GPU: as many splits as keep
-// one wave (tiles * ksplit <= SMs), each split at least 8 k steps long.
-int gemm_ksplit(int M, int K, int N, int sms) {
-    const int64_t tiles = (int64_t)gemm_mtiles(M) * gemm_ntiles(N);
-    if (tiles >= sms) return 1;
+size_t gemm_smem(int nb) { return (size_t)kGemmFixedSmem + 512 + (size_t)(nb + 1) * 4; }
+
+// Grid shape: whole waves of tiles (one tile per CTA), then the remaining
+// tiles with their k range split so that they fill one more wave (each split
+// at least eight 64-row steps).  Few tiles (small M) means all are split.
+struct GemmGrid {
+    int64_t tiles, full, rest;
+    int ksplit;
+    int64_t grid() const { return full + rest * ksplit; }
+};
+
+GemmGrid gemm_grid(int M, int K, int N, int sms) {
+    GemmGrid g;
+    g.tiles = (int64_t)gemm_mtiles(M) * gemm_ntiles(N);
+    g.full = g.tiles / sms * sms;
+    g.rest = g.tiles - g.full;
     const int nk = (K + kGemmBK - 1) / kGemmBK;
-    return (int)std::max<int64_t>(1, std::min<int64_t>(sms / tiles, nk / 8));
+    g.ksplit = g.rest ? (int)std::max<int64_t>(1, std::min<int64_t>(sms / g.rest, nk / 8)) : 1;
+    if (g.ksplit == 1) {  // nothing to split: every tile whole
+        g.full = g.tiles;
+        g.rest = 0;
+    }
+    return g;
 }
 
 // Workspace: [x_p fp16 M x K][row shifts int32 M][tickets][fp32 partial tiles].
@@ -384,16 +400,14 @@ struct GemmWs {
 };
 
 GemmWs gemm_ws_layout(int M, int K, int N, int sms) {
-    const int64_t tiles = (int64_t)gemm_mtiles(M) * gemm_ntiles(N);
-    const int ks = gemm_ksplit(M, K, N, sms);
+    const GemmGrid gg = gemm_grid(M, K, N, sms);
     GemmWs w;
     w.xshift = align_up((size_t)M * K * 2, 256);
     w.tickets = w.xshift + align_up((size_t)M * 4, 256);
-    w.partial = w.tickets + align_up((size_t)tiles * 4, 256);
-    w.total = w.partial + (ks > 1 ? (size_t)tiles * ks * kGemmBM * kGemmBN * 4 : 0);
+    w.partial = w.tickets + align_up((size_t)gg.tiles * 4, 256);
+    w.total = w.partial + (size_t)gg.rest * kGemmBM * kGemmBN * 4;
     return w;
 }
-size_t gemm_smem(int nb) { return (size_t)kGemmFixedSmem + 512 + (size_t)(nb + 1) * 4; }
 
 int make_gemm_maps(const void* xp, int x_dtype, int M, int K, const uint32_t* qw, int64_t qw_rows, int N,
                    GemmMaps* maps) {
@@ -466,13 +480,15 @@ int run_gemm(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     p.K = K;
     p.N = N;
     p.nb = nb;
+    const GemmGrid gg = gemm_grid(M, K, N, dev->sms);
     p.mtiles = gemm_mtiles(M);
     p.ntiles = gemm_ntiles(N);
-    p.ksplit = gemm_ksplit(M, K, N, dev->sms);
+    p.full_tiles = (int)gg.full;
+    p.ksplit = gg.ksplit;
     p.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.tickets);
     p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.partial);
     p.x_bf16 = bf16;
-    const unsigned grid = (unsigned)((int64_t)p.mtiles * p.ntiles * p.ksplit);
+    const unsigned grid = (unsigned)gg.grid();
     gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(p, maps);
     return launch_status();
 }
@@ -620,8 +636,9 @@ int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out) {
         return QGEMM_OK;
     }
     if (out[0] == kPathGemm) {
-        out[1] = (int64_t)gemm_mtiles(M) * gemm_ntiles(N) * gemm_ksplit(M, K, N, sms);
-        out[2] = gemm_ksplit(M, K, N, sms);
+        const GemmGrid gg = gemm_grid(M, K, N, sms);
+        out[1] = gg.grid();
+        out[2] = gg.ksplit;
         out[3] = 1;
         out[4] = (int64_t)gemm_smem(K / kBlockRows);
         return QGEMM_OK;
