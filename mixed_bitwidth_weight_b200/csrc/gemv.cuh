@@ -201,12 +201,13 @@ QG_DEV void decode_group(const uint8_t* w0, uint32_t ta) {
     }
 }
 
-// Units are numbered t*ng + g.  A unit's cost is its word rows plus its scale
-// row, so the cost prefix of (t, g) is t*(W + ng) + offs[4g] + g, with W the
-// word rows of one tile.  CTA i owns the units whose prefix lies in
+// Units are numbered t*ng + g (ng units per tile of bpu blocks each; four
+// blocks = one 128-row group by default).  A unit's cost is its word rows plus
+// one, so the cost prefix of (t, g) is t*(W + ng) + offs[bpu*g] + g, with W
+// the word rows of one tile.  CTA i owns the units whose prefix lies in
 // [ceil(i*C/G), ceil((i+1)*C/G)), C = tiles * (W + ng).
 QG_DEV int64_t unit_start(int64_t i, int64_t G, int64_t C, int64_t W, int nb, int ng, int tiles,
-                          const int32_t* s_offs) {
+                          const int32_t* s_offs, int bpu = kGemvGroupBlocks) {
     if (i >= G) return (int64_t)tiles * ng;
     const int64_t Wt = W + ng;
     int64_t t, rem;
@@ -222,16 +223,17 @@ QG_DEV int64_t unit_start(int64_t i, int64_t G, int64_t C, int64_t W, int nb, in
     int lo = 0, hi = ng;  // first g in [0, ng] with offs[min(4g, nb)] + g >= rem
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (s_offs[min(mid * kGemvGroupBlocks, nb)] + mid >= rem) hi = mid; else lo = mid + 1;
+        if (s_offs[min(mid * bpu, nb)] + mid >= rem) hi = mid; else lo = mid + 1;
     }
     return t * ng + lo;  // lo == ng rolls over to the next tile's group 0
 }
 
 // CTA that owns unit u.
-QG_DEV int cta_of(int64_t u, int64_t G, int64_t C, int64_t W, int ng, const int32_t* s_offs) {
+QG_DEV int cta_of(int64_t u, int64_t G, int64_t C, int64_t W, int ng, const int32_t* s_offs,
+                  int bpu = kGemvGroupBlocks) {
     const int64_t t = u / ng;
     const int g = (int)(u - t * ng);
-    const int64_t pos = t * (W + ng) + s_offs[g * kGemvGroupBlocks] + g;
+    const int64_t pos = t * (W + ng) + s_offs[g * bpu] + g;
     if (C * G < (1ll << 32)) return (int)(((uint32_t)pos * (uint32_t)G) / (uint32_t)C);
     return (int)((pos * G) / C);
 }

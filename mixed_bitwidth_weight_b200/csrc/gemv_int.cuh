@@ -45,14 +45,17 @@ namespace qg {
 constexpr int kIntMaxM = 4;
 constexpr int kIntThreads = kGemvDecThreads + 32;
 constexpr int kIntRowBytes = 1024;   // one ring row: 256 words (a box row lands densely)
-constexpr int kIntBoxMaps = 6;       // tensor maps with box heights 1, 2, 4, ..., 32 rows
+constexpr int kIntBoxMaps = 7;       // tensor maps with box heights 1, 2, 4, ..., 64 rows
+constexpr int kIntUnitGroups = 2;    // 128-row groups per unit
+constexpr int kIntUnitBlocks = kIntUnitGroups * kGemvGroupBlocks;  // 8 blocks, 256 rows
 
 // Tensor maps over qw [qw_rows][N] uint32, box {256 columns, 2^i rows}.
 struct IntMaps {
     CUtensorMap box[kIntBoxMaps];
 };
 
-// Ring rows of a unit: scale row, word rows, activation records.
+// Ring rows of a unit: one row holding its two scale rows (512 B each), the
+// word rows, the activation records.
 __host__ __device__ constexpr int int_unit_rows(int wrows, int nblk, int rec_bytes) {
     return 1 + wrows + (nblk * rec_bytes + kIntRowBytes - 1) / kIntRowBytes;
 }
@@ -333,19 +336,21 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
         }
         return;
     }
+    // units: (tile, pair of groups) = 8 blocks; nu units per tile
+    const int nu = (nb + kIntUnitBlocks - 1) / kIntUnitBlocks;
     const int64_t W = s_offs[nb];
-    const int64_t C = (int64_t)p.tiles * (W + ng);
+    const int64_t C = (int64_t)p.tiles * (W + nu);
     const int64_t G = gridDim.x;
-    const int64_t u0 = unit_start(blockIdx.x, G, C, W, nb, ng, p.tiles, s_offs);
-    const int64_t u1 = unit_start(blockIdx.x + 1, G, C, W, nb, ng, p.tiles, s_offs);
+    const int64_t u0 = unit_start(blockIdx.x, G, C, W, nb, nu, p.tiles, s_offs, kIntUnitBlocks);
+    const int64_t u1 = unit_start(blockIdx.x + 1, G, C, W, nb, nu, p.tiles, s_offs, kIntUnitBlocks);
     const int nunits = (int)(u1 - u0);
     if (nunits <= 0) {
         if (tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
         return;
     }
-    const int t0 = (int)(u0 / ng), gf = (int)(u0 - (int64_t)t0 * ng);
+    const int t0 = (int)(u0 / nu), gf = (int)(u0 - (int64_t)t0 * nu);
     auto rows_of = [&](int gg) {
-        const int a = gg * kGemvGroupBlocks, bb = min(a + kGemvGroupBlocks, nb);
+        const int a = gg * kIntUnitBlocks, bb = min(a + kIntUnitBlocks, nb);
         return int_unit_rows(s_offs[bb] - s_offs[a], bb - a, REC);
     };
 
@@ -359,7 +364,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
     if (warp == kGemvDecWarps) {
         if (lane > 2) return;
         auto issue = [&](int k, int t, int g, int row) {
-            const int j0 = g * kGemvGroupBlocks, j1 = min(j0 + kGemvGroupBlocks, nb);
+            const int j0 = g * kIntUnitBlocks, j1 = min(j0 + kIntUnitBlocks, nb);
             const int r0 = s_offs[j0], wrows = s_offs[j1] - r0;
             uint64_t* bar = &s_full[k & (kGemvSlots - 1)];
             uint8_t* dst = s_ring + (size_t)row * kIntRowBytes;
@@ -375,8 +380,11 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                     }
             } else if (lane == 1) {
                 const int cols = min(kGemvTileCols, p.N - t * kGemvTileCols);
-                mbar_arrive_expect_tx(bar, (uint32_t)(cols * 2));
-                bulk_g2s(dst, p.scales + (size_t)g * p.N + (size_t)t * kGemvTileCols, (uint32_t)cols * 2, bar);
+                const int g0 = g * kIntUnitGroups, ngr = min(kIntUnitGroups, ng - g0);
+                mbar_arrive_expect_tx(bar, (uint32_t)(ngr * cols * 2));
+                for (int u = 0; u < ngr; ++u)
+                    bulk_g2s(dst + u * 512, p.scales + (size_t)(g0 + u) * p.N + (size_t)t * kGemvTileCols,
+                             (uint32_t)cols * 2, bar);
             } else {
                 const int nblk = j1 - j0;
                 mbar_arrive_expect_tx(bar, (uint32_t)(nblk * REC));
@@ -398,7 +406,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                 pp = p2;
                 tot = t2;
                 ++npre;
-                if (++gg == ng) gg = 0;
+                if (++gg == nu) gg = 0;
             }
         }
         int pos = 0;
@@ -407,7 +415,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
         for (int k = 0; k < npre; ++k) {
             const int row = ring_alloc(pos, total, rows_of(g), R);
             if (lane != 2) issue(k, t, g, row);
-            if (++g == ng) { g = 0; ++t; }
+            if (++g == nu) { g = 0; ++t; }
         }
         if (lane == 2) {
             asm volatile("griddepcontrol.wait;" ::: "memory");  // activation records come from xprep_int
@@ -415,7 +423,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
             int64_t tot = 0;
             for (int k = 0; k < npre; ++k) {
                 issue(k, tt, gg, ring_alloc(pp, tot, rows_of(gg), R));
-                if (++gg == ng) { gg = 0; ++tt; }
+                if (++gg == nu) { gg = 0; ++tt; }
             }
         }
         int pos_rel = 0;
@@ -428,7 +436,11 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
             int ppos = pos;
             int64_t ptotal = total;
             ring_alloc(ppos, ptotal, need, R);
-            while (k - k_rel >= kGemvSlots || ptotal - total_rel > R) {
+            // room: the unit's rows are free once everything allocated more
+            // than R rows earlier is released; an empty ring (k_rel == k) always
+            // has room, which also covers a unit whose skipped tail plus its own
+            // rows exceed R
+            while (k - k_rel >= kGemvSlots || (ptotal - total_rel > R && k_rel < k)) {
                 const bool w = mbar_wait(&s_empty[k_rel & (kGemvSlots - 1)], (uint32_t)((k_rel / kGemvSlots) & 1));
                 if (!__all_sync(0x7u, w)) {
                     ok = false;
@@ -436,11 +448,11 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                 }
                 ring_alloc(pos_rel, total_rel, rows_of(g_rel), R);
                 ++k_rel;
-                if (++g_rel == ng) g_rel = 0;
+                if (++g_rel == nu) g_rel = 0;
             }
             if (!ok) break;
             issue(k, t, g, ring_alloc(pos, total, need, R));
-            if (++g == ng) { g = 0; ++t; }
+            if (++g == nu) { g = 0; ++t; }
         }
         if (!ok) {
             s_misc[3] = 1;
@@ -451,7 +463,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
     }
 
     // =================================================== consumer warps 0-7
-    const int bi = warp >> 1;                 // block slot within the group
+    const int bi = warp >> 1;                 // block slot within each group of the unit
     const int col0 = (warp & 1) * 128 + lane * 4;
     float yacc[4][MP];
 #pragma unroll
@@ -471,9 +483,9 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                 for (int t = 0; t < MP; ++t) s_red[((bi - 1) * kGemvTileCols + col0 + q) * MP + t] = yacc[q][t];
         }
         named_bar_sync(1, kGemvDecThreads);
-        const int64_t ut0 = (int64_t)tt * ng;
-        const int first = cta_of(ut0, G, C, W, ng, s_offs);
-        const int last = cta_of(ut0 + ng - 1, G, C, W, ng, s_offs);
+        const int64_t ut0 = (int64_t)tt * nu;
+        const int first = cta_of(ut0, G, C, W, nu, s_offs, kIntUnitBlocks);
+        const int last = cta_of(ut0 + nu - 1, G, C, W, nu, s_offs, kIntUnitBlocks);
         const int ncol = p.N - tt * kGemvTileCols;
         if (bi == 0) {
 #pragma unroll
@@ -520,21 +532,23 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
 #pragma unroll
                 for (int tt = 0; tt < MP; ++tt) yacc[q][tt] = 0.f;
         }
-        const int j0 = g * kGemvGroupBlocks, j1 = min(j0 + kGemvGroupBlocks, nb);
-        const int nblk = j1 - j0;
+        const int j0 = g * kIntUnitBlocks, j1 = min(j0 + kIntUnitBlocks, nb);
         const int o0 = s_offs[j0];
         const int wrows = s_offs[j1] - o0;
-        const int row = ring_alloc(pos, total, int_unit_rows(wrows, nblk, REC), R);
+        const int row = ring_alloc(pos, total, int_unit_rows(wrows, j1 - j0, REC), R);
         const int slot = k & (kGemvSlots - 1);
         if (!aborted && (s_misc[3] || !mbar_wait(&s_full[slot], (uint32_t)((k / kGemvSlots) & 1)))) {
             aborted = true;
             s_misc[3] = 1;
         }
-        if (!aborted && bi < nblk) {
-            const int j = j0 + bi;
+        const uint8_t* ub = s_ring + (size_t)row * kIntRowBytes;
+#pragma unroll 1
+        for (int gi = 0; gi < kIntUnitGroups; ++gi) {
+            const int bs = gi * kGemvGroupBlocks + bi;  // block slot within the unit
+            const int j = j0 + bs;
+            if (aborted || j >= j1) continue;
             const int b = s_offs[j + 1] - s_offs[j];
-            const uint8_t* ub = s_ring + (size_t)row * kIntRowBytes;
-            const uint8_t* rec = ub + (size_t)(1 + wrows) * kIntRowBytes + bi * REC;
+            const uint8_t* rec = ub + (size_t)(1 + wrows) * kIntRowBytes + bs * REC;
             uint32_t xp[MP][16];
             int32_t acc[4][MP];
 #pragma unroll
@@ -560,7 +574,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                 case 6: block_dp2a<6, MP>(wb, xp, acc); break;
                 default: block_dp2a<8, MP>(wb, xp, acc); break;
             }
-            const uint2 sv = *reinterpret_cast<const uint2*>(ub + col0 * 2);
+            const uint2 sv = *reinterpret_cast<const uint2*>(ub + gi * 512 + col0 * 2);
             float sc[4];
             sc[0] = __low2float(*reinterpret_cast<const __half2*>(&sv.x));
             sc[1] = __high2float(*reinterpret_cast<const __half2*>(&sv.x));
@@ -577,7 +591,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
         }
         __syncwarp();
         if (lane == 0 && !aborted) mbar_arrive(&s_empty[slot]);
-        if (++g == ng) { g = 0; ++t; }
+        if (++g == nu) { g = 0; ++t; }
     }
     flush(t_prev);
 
@@ -593,9 +607,9 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
             const int pt = i ? pend1 : pend0;
             int is_last = 0;
             if (pt >= 0 && !s_misc[3]) {
-                const int64_t ut0 = (int64_t)pt * ng;
-                const int first = cta_of(ut0, G, C, W, ng, s_offs);
-                const int last = cta_of(ut0 + ng - 1, G, C, W, ng, s_offs);
+                const int64_t ut0 = (int64_t)pt * nu;
+                const int first = cta_of(ut0, G, C, W, nu, s_offs, kIntUnitBlocks);
+                const int last = cta_of(ut0 + nu - 1, G, C, W, nu, s_offs, kIntUnitBlocks);
                 is_last = (atomicAdd(&p.tickets[pt], 1) == last - first);
             }
             s_misc[1 + i] = is_last;
@@ -607,11 +621,11 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
         if (!s_misc[1 + i]) continue;
         __threadfence();
         const int tt = i ? pend1 : pend0;
-        const int64_t ut0 = (int64_t)tt * ng;
-        const int first = cta_of(ut0, G, C, W, ng, s_offs);
-        const int last = cta_of(ut0 + ng - 1, G, C, W, ng, s_offs);
+        const int64_t ut0 = (int64_t)tt * nu;
+        const int first = cta_of(ut0, G, C, W, nu, s_offs, kIntUnitBlocks);
+        const int last = cta_of(ut0 + nu - 1, G, C, W, nu, s_offs, kIntUnitBlocks);
         const int ncol = p.N - tt * kGemvTileCols;
-        const bool first_before = (tt > 0) && cta_of(ut0 - 1, G, C, W, ng, s_offs) == first;
+        const bool first_before = (tt > 0) && cta_of(ut0 - 1, G, C, W, nu, s_offs, kIntUnitBlocks) == first;
         for (int e = tid; e < M * kGemvTileCols; e += kGemvDecThreads) {
             const int tok = e / kGemvTileCols, cl = e - tok * kGemvTileCols;
             if (cl >= ncol) continue;

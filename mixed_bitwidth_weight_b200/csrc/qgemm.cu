@@ -270,9 +270,11 @@ int plan_int(int M, int K, int N, int64_t qw_rows, int sms, GemvPlan* plan, int*
     const int nb = K / kBlockRows;
     const int mp = int_mp(M);
     const int cps = int_ctas_per_sm(mp);
-    const int64_t U = (int64_t)gemv_tiles(N) * gemv_groups(K);
-    const int64_t C = (int64_t)gemv_tiles(N) * (qw_rows + gemv_groups(K));
-    const int64_t gcap = std::max<int64_t>(1, C / (8 * kGemvGroupBlocks + 2));
+    // units of two 128-row groups: cost = word rows + 1, at most 8 * 8 + 1
+    const int64_t nu = (nb + kIntUnitBlocks - 1) / kIntUnitBlocks;
+    const int64_t U = (int64_t)gemv_tiles(N) * nu;
+    const int64_t C = (int64_t)gemv_tiles(N) * (qw_rows + nu);
+    const int64_t gcap = std::max<int64_t>(1, C / (8 * kIntUnitBlocks + 2));
     const int64_t G = std::min<int64_t>(std::min<int64_t>(U, gcap), (int64_t)cps * sms);
     const size_t fixed = int_fixed_smem(nb, mp);
     const size_t budget = (size_t)(cps == 2 ? 113 : 227) * 1024;

@@ -20,14 +20,15 @@ from tests import problems as P
 TILE = 256
 
 
-def replay(offs, tiles, G):
-    """The kernel's split: units are (tile, 128-row group), numbered t*ng + g; a
-    unit costs its word rows plus one scale row."""
+def replay(offs, tiles, G, bpu=4):
+    """The kernel's split: units are (tile, bpu blocks), numbered t*ng + g; a
+    unit costs its word rows plus one.  bpu = 4 (one 128-row group) for the
+    tensor-core GEMV, 8 (two groups) for the integer GEMV."""
     nb = len(offs) - 1
-    ng = (nb + 3) // 4
+    ng = (nb + bpu - 1) // bpu
     Wt = int(offs[-1]) + ng
     C = tiles * Wt
-    goffs = [int(offs[min(4 * g, nb)]) + g for g in range(ng + 1)]
+    goffs = [int(offs[min(bpu * g, nb)]) + g for g in range(ng + 1)]
 
     def unit_start(i):
         if i >= G:
@@ -81,7 +82,8 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     # resident CTAs fit the SM's 228 KB (1 KB reserved per CTA)
     assert cps * (plan["smem"] + 1024) <= 228 * 1024
     assert plan["ring"] >= 80
-    starts, cta_of, ng = replay(offs, tiles, G)
+    bpu = 8 if integer else 4
+    starts, cta_of, ng = replay(offs, tiles, G, bpu)
     assert starts[0] == 0 and starts[-1] == tiles * ng
     assert all(a <= b for a, b in zip(starts, starts[1:]))
     ws = q.qgemm_workspace_bytes(M, K, N)
@@ -104,6 +106,45 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
         assert owners == expect, t
     # a unit (scale row, a group's word rows, activation records) fits the ring
     row_bytes = 1024 if integer else 1056
-    need = max(1 + int(offs[min(4 * g + 4, nb)] - offs[4 * g]) + -(-min(4, nb - 4 * g) * rec // row_bytes)
+    need = max(1 + int(offs[min(bpu * g + bpu, nb)] - offs[bpu * g]) + -(-min(bpu, nb - bpu * g) * rec // row_bytes)
                for g in range(ng))
     assert need <= plan["ring"]
+
+
+def ring_progress(rows_seq, R, slots=16):
+    """Replay the producer's admission rule with the consumers releasing units
+    in order only when asked: every unit must be admitted at the latest once all
+    earlier units are released (no wait that can never end)."""
+    def alloc(pos, total, need):
+        if pos + need > R:
+            total += R - pos
+            pos = 0
+        return pos, pos + need, total + need
+
+    pos = pos_rel = 0
+    total = total_rel = 0
+    k_rel = 0
+    for k, need in enumerate(rows_seq):
+        assert need <= R
+        _, ppos, ptotal = alloc(pos, total, need)
+        while k - k_rel >= slots or (ptotal - total_rel > R and k_rel < k):
+            _, pos_rel, total_rel = alloc(pos_rel, total_rel, rows_seq[k_rel])
+            k_rel += 1
+        _, pos, total = alloc(pos, total, need)
+
+
+@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("case", shapes(), ids=lambda c: f"{c[0]}-{c[1]}x{c[2]}")
+def test_integer_gemv_ring_always_admits(case, M):
+    name, K, N, bits = case
+    offs = W.offsets(bits)
+    nb = K // 32
+    plan = q.qgemm_plan_info(M, K, N, int(offs[-1]))
+    mp = 1 if M == 1 else 2 if M == 2 else 4
+    rec = (72 * mp + 15) // 16 * 16
+    nu = (nb + 7) // 8
+    rows = [1 + int(offs[min(8 * g + 8, nb)] - offs[8 * g]) + -(-min(8, nb - 8 * g) * rec // 1024)
+            for g in range(nu)]
+    seq = rows * 3                      # a CTA range can run over several tiles
+    for start in range(0, nu, max(1, nu // 8)):
+        ring_progress(seq[start:start + 2 * nu], plan["ring"])
