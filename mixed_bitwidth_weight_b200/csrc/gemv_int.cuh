@@ -213,7 +213,11 @@ QG_DEV void block_dp2a(const uint8_t* w, const uint32_t (&xp)[MP][16], int32_t (
 // groups per CTA.  Group maximum -> e; x_int = rint(x * 2^e); zsum =
 // z * sum of the block's x_int.
 __global__ void __launch_bounds__(256) xprep_int_kernel(const IntPrepParams p) {
+    // launched as a programmatic dependent of the previous grid in the stream
+    // (a decode GEMV, say): x may be that grid's output and the records below
+    // may still be read by it, so wait for it before any load of x or store
     asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ int s_gmax[2][kIntMaxM];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gl = warp >> 2;
     if (threadIdx.x < 2 * kIntMaxM) s_gmax[threadIdx.x / kIntMaxM][threadIdx.x % kIntMaxM] = 0;
@@ -280,6 +284,9 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nb = p.nb, ng = p.ng, M = p.M;
+    // the next call's activation kernel may start during this grid's tail; it
+    // waits for this grid's completion before it touches x or the workspace
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;");
 
     int32_t* s_offs = reinterpret_cast<int32_t*>(smem);
     size_t o = ((size_t)(nb + 1) * 4 + 15) & ~(size_t)15;

@@ -337,8 +337,23 @@ int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t
     xp.nb = nb;
     xp.mp = mp;
     xp.x_bf16 = (x_dtype == QGEMM_BF16);
-    xprep_int_kernel<<<(nb + 7) / 8, 256, 0, stream>>>(xp);
-    if ((st = launch_status()) != QGEMM_OK) return st;
+    {
+        // programmatic dependent of the previous grid (it waits for it on the
+        // device), so its launch overlaps that grid's tail
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((nb + 7) / 8);
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, xprep_int_kernel, xp) != cudaSuccess) {
+            cudaGetLastError();
+            return QGEMM_ERR_CUDA;
+        }
+    }
 
     IntParams p;
     p.rec = xp.rec;
