@@ -46,6 +46,7 @@ constexpr int kGemmRBytes = (kGemmRawRows + 1) * 1024;   // scale row + word row
 constexpr int kGemmDecWarps = 8;
 constexpr int kGemmThreads = 64 + kGemmDecWarps * 32;
 constexpr int kGemmBoxMaps = 5;                          // word boxes of 1, 2, 4, 8, 16 rows
+constexpr int kGemmMaxSplit = 4;                         // k splits of one tile, at most
 constexpr int kGemmFixedSmem =
     kGemmAStages * kGemmABytes + kGemmBStages * kGemmBBytes + kGemmRStages * kGemmRBytes + 1024;
 
@@ -62,7 +63,7 @@ struct GemmParams {
     int64_t qw_rows;
     __half* y;
     int* tickets;      // [tiles] (split tiles only)
-    float* partial;    // [split tiles][256][256] fp32 sums, zero between calls
+    float* partial;    // [split tiles][ksplit][256][256] fp32 partial sums
     int M, K, N, nb, mtiles, ntiles, x_bf16;
     int full_tiles;    // tiles done whole, one per CTA (whole waves of the grid)
     int ksplit;        // k splits of each remaining tile (the last wave)
@@ -420,47 +421,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         };
         if (ok && (h == 0 || two)) {
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + h * kGemmBN;
-            float* acc = p.partial + (size_t)(tile - full) * (kGemmBM * kGemmBN) + (size_t)rl * kGemmBN;
+            float* part =
+                p.partial + ((size_t)(tile - full) * nsplit + ks) * (kGemmBM * kGemmBN) + (size_t)rl * kGemmBN;
 #pragma unroll 1
             for (int c = 0; c < kGemmBN; c += 16) {
                 float v[16];
                 tmem_ld16(taddr + c, v);
                 if (nsplit == 1) {
                     if (row < p.M && n0 + c < p.N) store_y(row, c, v, g1, g2);
-                } else if (row < p.M) {
-                    // fire-and-forget vector reductions into the tile's fp32 sum
-                    // (only columns of y: the accumulator outside stays zero)
+                } else {
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        if (n0 + c + 4 * u < p.N)
-                            atomicAdd(reinterpret_cast<float4*>(acc + c + 4 * u),
-                                      make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]));
+                        __stcg(reinterpret_cast<float4*>(part + c + 4 * u),
+                               make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]));
                 }
             }
         }
         if (nsplit > 1) {
-            // the last of the tile's nsplit CTAs converts the sum to y and
-            // leaves the accumulator at zero for the next call
+            // the last of the tile's nsplit CTAs adds the partial sums in split
+            // order (the same bits on every call), one float4 per thread step
             __threadfence();
             named_bar_sync(1, kGemmDecWarps * 32);
             if (tid == 64) s_misc[3] = (ok && !s_misc[1]) ? (atomicAdd(&p.tickets[tile], 1) == nsplit - 1) : 0;
             named_bar_sync(1, kGemmDecWarps * 32);
             if (s_misc[3]) {
                 __threadfence();
-                float4* acc4 = reinterpret_cast<float4*>(p.partial + (size_t)(tile - full) * (kGemmBM * kGemmBN));
+                const float4* base4 =
+                    reinterpret_cast<const float4*>(p.partial + (size_t)(tile - full) * nsplit * (kGemmBM * kGemmBN));
                 const int t = tid - 64;
-#pragma unroll 4
-                for (int f = t; f < kGemmBM * kGemmBN / 4; f += kGemmDecWarps * 32) {
+                const int rows = min(kGemmBM, p.M - m0);
+#pragma unroll 2
+                for (int f = t; f < rows * (kGemmBN / 4); f += kGemmDecWarps * 32) {
                     const int r2 = f / (kGemmBN / 4), c4 = (f % (kGemmBN / 4)) * 4;
+                    if (n0 + c4 >= p.N) continue;
+                    float4 a[kGemmMaxSplit];
+#pragma unroll
+                    for (int kq = 0; kq < kGemmMaxSplit; ++kq)
+                        if (kq < nsplit) a[kq] = __ldcg(base4 + (size_t)kq * (kGemmBM * kGemmBN / 4) + f);
+                    float4 sum = a[0];
+#pragma unroll
+                    for (int kq = 1; kq < kGemmMaxSplit; ++kq)
+                        if (kq < nsplit) {
+                            sum.x += a[kq].x;
+                            sum.y += a[kq].y;
+                            sum.z += a[kq].z;
+                            sum.w += a[kq].w;
+                        }
                     const int row2 = m0 + r2;
-                    if (row2 >= p.M || n0 + c4 >= p.N) continue;
-                    const float4 a = __ldcg(acc4 + f);
-                    __stcg(acc4 + f, make_float4(0.f, 0.f, 0.f, 0.f));
                     const int sh2 = p.x_bf16 ? p.xshift[row2] : 0;
                     const float s1 = __int_as_float((127 + sh2 / 2) << 23);
                     const float s2 = __int_as_float((127 + (sh2 - sh2 / 2)) << 23);
-                    const __half2 lo = __floats2half2_rn(a.x * s1 * s2, a.y * s1 * s2);
-                    const __half2 hi = __floats2half2_rn(a.z * s1 * s2, a.w * s1 * s2);
+                    const __half2 lo = __floats2half2_rn(sum.x * s1 * s2, sum.y * s1 * s2);
+                    const __half2 hi = __floats2half2_rn(sum.z * s1 * s2, sum.w * s1 * s2);
                     *reinterpret_cast<uint2*>(p.y + (size_t)row2 * p.N + n0 + c4) =
                         make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
                 }

@@ -245,6 +245,7 @@ __global__ void __launch_bounds__(256) xprep_int_kernel(const IntPrepParams p) {
     __syncthreads();
 #pragma unroll
     for (int m = 0; m < kIntMaxM; ++m) {
+        if (m >= p.M) break;  // uniform over the block
         int a = __float_as_int(fabsf(v[m]));
         if (a >= 0x7F800000) a = 0x7F7FFFFF;  // inf / nan: saturate the scale choice
 #pragma unroll
@@ -281,6 +282,7 @@ template <int MP>
 __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
     gemv_int_kernel(const IntParams p, const __grid_constant__ IntMaps maps) {
     constexpr int REC = int_rec_bytes(MP);
+    constexpr int TP = MP < 4 ? MP : 4;  // tokens per pass
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nb = p.nb, ng = p.ng, M = p.M;
@@ -556,44 +558,49 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
             if (aborted || j >= j1) continue;
             const int b = s_offs[j + 1] - s_offs[j];
             const uint8_t* rec = ub + (size_t)(1 + wrows) * kIntRowBytes + bs * REC;
-            uint32_t xp[MP][16];
-            int32_t acc[4][MP];
-#pragma unroll
-            for (int tt = 0; tt < MP; ++tt) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint4 v = reinterpret_cast<const uint4*>(rec + tt * 64)[i];
-                    xp[tt][4 * i] = v.x;
-                    xp[tt][4 * i + 1] = v.y;
-                    xp[tt][4 * i + 2] = v.z;
-                    xp[tt][4 * i + 3] = v.w;
-                }
-                const int32_t zs = reinterpret_cast<const int32_t*>(rec + 64 * MP)[tt];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc[q][tt] = -zs;
-            }
             const uint8_t* wb = ub + (size_t)(1 + s_offs[j] - o0) * kIntRowBytes + col0 * 4;
-            switch (b) {
-                case 2: block_dp2a<2, MP>(wb, xp, acc); break;
-                case 3: block_dp2a<3, MP>(wb, xp, acc); break;
-                case 4: block_dp2a<4, MP>(wb, xp, acc); break;
-                case 5: block_dp2a<5, MP>(wb, xp, acc); break;
-                case 6: block_dp2a<6, MP>(wb, xp, acc); break;
-                default: block_dp2a<8, MP>(wb, xp, acc); break;
-            }
             const uint2 sv = *reinterpret_cast<const uint2*>(ub + gi * 512 + col0 * 2);
             float sc[4];
             sc[0] = __low2float(*reinterpret_cast<const __half2*>(&sv.x));
             sc[1] = __high2float(*reinterpret_cast<const __half2*>(&sv.x));
             sc[2] = __low2float(*reinterpret_cast<const __half2*>(&sv.y));
             sc[3] = __high2float(*reinterpret_cast<const __half2*>(&sv.y));
+            // tokens in passes of up to four (registers); each pass re-reads the
+            // block's word rows from shared memory
 #pragma unroll
-            for (int tt = 0; tt < MP; ++tt) {
-                const int e = reinterpret_cast<const int32_t*>(rec + 68 * MP)[tt] + int_acc_shift(b);
-                const int e1 = e / 2, e2 = e - e / 2;
-                const float f1 = __int_as_float((127 - e1) << 23), f2 = __int_as_float((127 - e2) << 23);
+            for (int ps = 0; ps < MP / TP; ++ps) {
+                uint32_t xp[TP][16];
+                int32_t acc[4][TP];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) yacc[q][tt] += ((float)acc[q][tt] * sc[q]) * f1 * f2;
+                for (int tt = 0; tt < TP; ++tt) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 v = reinterpret_cast<const uint4*>(rec + (ps * TP + tt) * 64)[i];
+                        xp[tt][4 * i] = v.x;
+                        xp[tt][4 * i + 1] = v.y;
+                        xp[tt][4 * i + 2] = v.z;
+                        xp[tt][4 * i + 3] = v.w;
+                    }
+                    const int32_t zs = reinterpret_cast<const int32_t*>(rec + 64 * MP)[ps * TP + tt];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[q][tt] = -zs;
+                }
+                switch (b) {
+                    case 2: block_dp2a<2, TP>(wb, xp, acc); break;
+                    case 3: block_dp2a<3, TP>(wb, xp, acc); break;
+                    case 4: block_dp2a<4, TP>(wb, xp, acc); break;
+                    case 5: block_dp2a<5, TP>(wb, xp, acc); break;
+                    case 6: block_dp2a<6, TP>(wb, xp, acc); break;
+                    default: block_dp2a<8, TP>(wb, xp, acc); break;
+                }
+#pragma unroll
+                for (int tt = 0; tt < TP; ++tt) {
+                    const int e = reinterpret_cast<const int32_t*>(rec + 68 * MP)[ps * TP + tt] + int_acc_shift(b);
+                    const int e1 = e / 2, e2 = e - e / 2;
+                    const float f1 = __int_as_float((127 - e1) << 23), f2 = __int_as_float((127 - e2) << 23);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) yacc[q][ps * TP + tt] += ((float)acc[q][tt] * sc[q]) * f1 * f2;
+                }
             }
         }
         __syncwarp();

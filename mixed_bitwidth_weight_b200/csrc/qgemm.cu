@@ -200,6 +200,11 @@ int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
 
 // ----------------------------------------------------------- integer GEMV
 constexpr int kPathGemvInt = 0, kPathGemvTc = 1, kPathGemm = 2;
+// M served by the integer GEMV (measured: above four tokens the tensor-core
+// GEMV is faster)
+constexpr int kIntPathMaxM = 4;
+// M served by the allocation-free decode entry point
+constexpr int kNoAllocMaxM = 4;
 
 int int_mp(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
 int int_ctas_per_sm(int mp) { return mp <= 2 ? 2 : 1; }
@@ -390,7 +395,8 @@ size_t gemm_smem(int nb) { return (size_t)kGemmFixedSmem + 512 + (size_t)(nb + 1
 
 // Grid shape: whole waves of tiles (one tile per CTA), then the remaining
 // tiles with their k range split so that they fill one more wave (each split
-// at least eight 64-row steps).  Few tiles (small M) means all are split.
+// at least eight 64-row steps, at most kGemmMaxSplit splits).  Few tiles
+// (small M) means all are split.
 struct GemmGrid {
     int64_t tiles, full, rest;
     int ksplit;
@@ -403,7 +409,9 @@ GemmGrid gemm_grid(int M, int K, int N, int sms) {
     g.full = g.tiles / sms * sms;
     g.rest = g.tiles - g.full;
     const int nk = (K + kGemmBK - 1) / kGemmBK;
-    g.ksplit = g.rest ? (int)std::max<int64_t>(1, std::min<int64_t>(sms / g.rest, nk / 8)) : 1;
+    g.ksplit = g.rest ? (int)std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(sms / g.rest, nk / 8),
+                                                                    kGemmMaxSplit))
+                      : 1;
     if (g.ksplit == 1) {  // nothing to split: every tile whole
         g.full = g.tiles;
         g.rest = 0;
@@ -422,7 +430,7 @@ GemmWs gemm_ws_layout(int M, int K, int N, int sms) {
     w.xshift = align_up((size_t)M * K * 2, 256);
     w.tickets = w.xshift + align_up((size_t)M * 4, 256);
     w.partial = w.tickets + align_up((size_t)gg.tiles * 4, 256);
-    w.total = w.partial + (size_t)gg.rest * kGemmBM * kGemmBN * 4;
+    w.total = w.partial + (size_t)gg.rest * gg.ksplit * kGemmBM * kGemmBN * 4;
     return w;
 }
 
@@ -609,7 +617,7 @@ size_t qgemm_scale_bytes(int K, int N) {
 int qgemm_path_for(int M, int K, int N) {
     (void)K;
     (void)N;
-    return M <= kIntMaxM ? kPathGemvInt : M <= 16 ? kPathGemvTc : kPathGemm;
+    return M <= kIntPathMaxM ? kPathGemvInt : M <= 16 ? kPathGemvTc : kPathGemm;
 }
 
 size_t qgemm_workspace_bytes(int M, int K, int N) {
@@ -737,7 +745,7 @@ int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm, co
     if (x_dtype != QGEMM_F16 && x_dtype != QGEMM_BF16) return QGEMM_ERR_DTYPE;
     int st = check_shape(K, N);
     if (st != QGEMM_OK) return st;
-    if (M < 1 || M > kIntMaxM) return QGEMM_ERR_SHAPE;
+    if (M < 1 || M > kNoAllocMaxM) return QGEMM_ERR_SHAPE;
     if ((st = check_rows(K, qw_rows)) != QGEMM_OK) return st;
     if (!aligned16(d_x) || !aligned16(d_perm) || !aligned16(d_qw) || !aligned16(d_scales) || !aligned16(d_y))
         return QGEMM_ERR_ALIGN;

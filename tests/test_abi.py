@@ -91,6 +91,7 @@ def test_workspace_and_sizes():
     assert q.qgemm_path_for(4, 8192, 8192) == 0
     assert q.qgemm_path_for(5, 8192, 8192) == 1      # tensor-core GEMV
     assert q.qgemm_path_for(16, 8192, 8192) == 1
+    assert q.qgemm_path_for(17, 8192, 8192) == 2
     assert q.qgemm_path_for(2048, 8192, 8192) == 2   # GEMM
 
 
@@ -129,14 +130,13 @@ def test_gemm_plan_and_workspace():
     the workspace, shared memory within the 227 KB a CTA may use up to K = 65536."""
     plan = q.qgemm_plan_info(2048, 8192, 28672, 992)
     assert plan["path"] == 2
-    # 896 tiles: six whole waves of 148, the last 8 tiles split 16 ways
-    # (148 // 8 = 18, capped at 128 k steps / 8)
-    assert plan["ring"] == 16 and plan["grid"] == 888 + 8 * 16
+    # 896 tiles: six whole waves of 148, the last 8 tiles split 4 ways (the cap)
+    assert plan["ring"] == 4 and plan["grid"] == 888 + 8 * 4
     assert plan["smem"] <= 227 * 1024
-    assert q.qgemm_workspace_bytes(2048, 8192, 28672) >= 2048 * 8192 * 2 + 8 * 256 * 256 * 4
+    assert q.qgemm_workspace_bytes(2048, 8192, 28672) >= 2048 * 8192 * 2 + 8 * 4 * 256 * 256 * 4
     big = q.qgemm_plan_info(17, 65536, 8, 2 * 2048)
     assert big["smem"] <= 227 * 1024
-    # one output tile: k is split so that the SMs have work, 8+ k steps each
+    # one output tile: k is split (at most 4 ways), 8+ k steps each
     ks = big["ring"]
-    assert 1 < ks <= 148 and big["grid"] == ks and (65536 // 64) // ks >= 8
-    assert q.qgemm_workspace_bytes(17, 65536, 8) >= 17 * 65536 * 2 + 256 * 256 * 4
+    assert ks == 4 and big["grid"] == ks
+    assert q.qgemm_workspace_bytes(17, 65536, 8) >= 17 * 65536 * 2 + ks * 256 * 256 * 4

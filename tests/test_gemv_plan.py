@@ -68,12 +68,12 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     rows = int(offs[-1])
     tiles = (N + TILE - 1) // TILE
     plan = q.qgemm_plan_info(M, K, N, rows)
-    integer = M <= 4
-    assert plan["path"] == (0 if integer else 1)
+    integer = plan["path"] == 0
+    assert plan["path"] in (0, 1)
     G = plan["grid"]
     cps = plan["ctas_per_sm"]
     if integer:
-        mp = 1 if M == 1 else 2 if M == 2 else 4
+        mp = 1 if M == 1 else 2 if M == 2 else 4 if M <= 4 else 8 if M <= 8 else 16
         assert cps == (2 if mp <= 2 else 1)
     else:
         mp = 8 if M <= 8 else 16
@@ -133,14 +133,14 @@ def ring_progress(rows_seq, R, slots=16):
         _, pos, total = alloc(pos, total, need)
 
 
-@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("M", [1, 4, 16])
 @pytest.mark.parametrize("case", shapes(), ids=lambda c: f"{c[0]}-{c[1]}x{c[2]}")
 def test_integer_gemv_ring_always_admits(case, M):
     name, K, N, bits = case
     offs = W.offsets(bits)
     nb = K // 32
     plan = q.qgemm_plan_info(M, K, N, int(offs[-1]))
-    mp = 1 if M == 1 else 2 if M == 2 else 4
+    mp = 1 if M == 1 else 2 if M == 2 else 4 if M <= 4 else 8 if M <= 8 else 16
     rec = (72 * mp + 15) // 16 * 16
     nu = (nb + 7) // 8
     rows = [1 + int(offs[min(8 * g + 8, nb)] - offs[8 * g]) + -(-min(8, nb - 8 * g) * rec // 1024)

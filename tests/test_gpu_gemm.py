@@ -51,24 +51,14 @@ def test_gemm_parity(q, M, K, N, x_dtype):
 
 @pytest.mark.parametrize("M,K,N", [(64, 8192, 512), (200, 4096, 256), (33, 2048, 1032)])
 def test_gemm_split_k(q, M, K, N):
-    """Few output tiles: k is split across CTAs, which add their partial sums
-    into an fp32 tile; the last one writes y and zeroes the tile again, so a
-    second call on the same workspace is as good as the first."""
+    """Few output tiles: k is split across CTAs; the last one adds the partial
+    sums in split order (the same bits on every call, tickets back to zero)."""
     plan = q.qgemm_plan_info(M, K, N, int(P.make(K, 8, kind="shuffled", seed=1)["offs"][-1]))
     assert plan["ring"] > 1                       # k splits
     pr = P.make(K, N, M=M, kind="shuffled", seed=M + N, x_dtype=torch.bfloat16)
-    g = P.to_gpu(pr)
-    ws = q.workspace(M, K, N)
-    yr = P.ref_y(pr)
-    for _ in range(2):
-        y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
-        q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, ws)
-        torch.cuda.synchronize()
-        P.check_close(y, yr)
-    assert int(ws.abs().sum()) > 0                   # x_p lives there
-    plan_bytes = q.qgemm_workspace_bytes(M, K, N)
-    acc = ws[plan_bytes - 256 * 256 * 4:].view(torch.float32)
-    assert int((acc != 0).sum()) == 0                # the last split tile's sum is back to zero
+    a = run(q, pr)
+    P.check_close(a, P.ref_y(pr))
+    assert torch.equal(a, run(q, pr))
 
 
 @pytest.mark.parametrize("kind", ["u2", "u3", "u4", "u5", "u6", "u8", "sorted"])
@@ -100,8 +90,7 @@ def test_gemm_subnormal_scales(q):
 
 def test_gemm_whole_tiles_deterministic(q):
     """At least one whole wave of tiles: no k split, a fixed summation order,
-    the same bits on every call (split tiles add partial sums with atomics
-    and may differ in the last fp32 bits)."""
+    the same bits on every call."""
     M, K, N = 256, 512, 148 * 256
     plan = q.qgemm_plan_info(M, K, N, int(P.make(K, 8, kind="shuffled", seed=4)["offs"][-1]))
     assert plan["ring"] == 1
