@@ -615,9 +615,16 @@ size_t qgemm_scale_bytes(int K, int N) {
 }
 
 int qgemm_path_for(int M, int K, int N) {
-    (void)K;
-    (void)N;
-    return M <= kIntPathMaxM ? kPathGemvInt : M <= 16 ? kPathGemvTc : kPathGemm;
+    if (M <= kIntPathMaxM) return kPathGemvInt;
+    if (M > 16) return kPathGemm;
+    // 5..16 rows: the tensor-core GEMV, except from 12 rows on when the GEMM
+    // splits k across the SMs (few output tiles), where it measured faster
+    if (M >= 12 && K > 0 && N > 0) {
+        DeviceInfo* dev = nullptr;
+        const int sms = (current_device_info(&dev) == QGEMM_OK) ? dev->sms : 148;
+        if (gemm_grid(M, K, N, sms).ksplit > 1) return kPathGemm;
+    }
+    return kPathGemvTc;
 }
 
 size_t qgemm_workspace_bytes(int M, int K, int N) {

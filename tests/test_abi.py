@@ -90,7 +90,9 @@ def test_workspace_and_sizes():
     assert q.qgemm_path_for(1, 8192, 8192) == 0      # integer GEMV
     assert q.qgemm_path_for(4, 8192, 8192) == 0
     assert q.qgemm_path_for(5, 8192, 8192) == 1      # tensor-core GEMV
-    assert q.qgemm_path_for(16, 8192, 8192) == 1
+    assert q.qgemm_path_for(11, 8192, 8192) == 1
+    assert q.qgemm_path_for(12, 8192, 8192) == 2     # few tiles: the split-k GEMM
+    assert q.qgemm_path_for(16, 8192, 28672) == 1    # 112 tiles, no split: the GEMV
     assert q.qgemm_path_for(17, 8192, 8192) == 2
     assert q.qgemm_path_for(2048, 8192, 8192) == 2   # GEMM
 

