@@ -15,8 +15,8 @@
 //                  columns) and issues the MMAs from one thread:
 //                  tcgen05.mma kind::f16, M = 128, N = 256, K = 16, both
 //                  operands from shared memory;
-//     warps 2-9  - dequantise: thread n decodes the 64 codes of column n in
-//                  the step (two 32-row blocks, each at its own width) two
+//     warps 2-17 - dequantise: thread (n, k) decodes the 32 codes of column n
+//                  in block k of the step (each block at its own width) two
 //                  per instruction in fp16 pairs, forms w = (q - 2^(b-1)) * s
 //                  with one rounding (the bit-exact dequantised weight) and
 //                  writes row n of the B tile in the
@@ -43,7 +43,7 @@ constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;       // 32 KB
 constexpr int kGemmBBytes = kGemmBN * kGemmBK * 2;       // 32 KB
 constexpr int kGemmRawRows = 16;                         // word rows of two blocks, at most
 constexpr int kGemmRBytes = (kGemmRawRows + 1) * 1024;   // scale row + word rows
-constexpr int kGemmDecWarps = 8;
+constexpr int kGemmDecWarps = 16;                        // 2 blocks x 256 columns per k step
 constexpr int kGemmThreads = 64 + kGemmDecWarps * 32;
 constexpr int kGemmBoxMaps = 5;                          // word boxes of 1, 2, 4, 8, 16 rows
 constexpr int kGemmMaxSplit = 4;                         // k splits of one tile, at most
@@ -361,7 +361,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ================================================= dequant warps
-        const int n = tid - 64;                 // column within the tile
+        const int n = (tid - 64) & (kGemmBN - 1);  // column within the tile
+        const int blk = (tid - 64) >> 8;           // block of the k step (warps 2-9: 0, 10-17: 1)
         for (int i = 0; i < nk; ++i) {
             const int sr = i % kGemmRStages, sb = i % kGemmBStages;
             if (s_misc[1] || !mbar_wait(&r_full[sr], (uint32_t)((i / kGemmRStages) & 1)) ||
@@ -375,8 +376,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint8_t* brow = sB + sb * kGemmBBytes + n * 128;
             const int j0 = 2 * (kb + i);
             const int r0 = s_offs[j0];
-#pragma unroll
-            for (int blk = 0; blk < 2; ++blk) {
+            {
                 const int j = j0 + blk;
                 uint32_t out[16];
                 if (j < nb) {
@@ -403,7 +403,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ---- epilogue: TMEM -> y (fp16), or fp32 partial sums under split K
         const bool ok = mbar_wait(acc_full, 0) && !s_misc[1];
         tc_fence_after();
-        const int q = warp & 3, h = (warp - 2) >> 2;
+        // warp: TMEM lane quadrant warp % 4 (the only lanes it may access),
+        // accumulator (128-row half) h and 128-column half ch
+        const int q = warp & 3, sel = (warp - 2) >> 2, h = sel & 1, ch = sel >> 1;
         const int rl = h * 128 + q * 32 + lane;  // row within the tile
         const int row = m0 + rl;
         const int sh = (p.x_bf16 && row < p.M) ? p.xshift[row] : 0;
@@ -424,7 +426,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float* part =
                 p.partial + ((size_t)(tile - full) * nsplit + ks) * (kGemmBM * kGemmBN) + (size_t)rl * kGemmBN;
 #pragma unroll 1
-            for (int c = 0; c < kGemmBN; c += 16) {
+            for (int c = ch * (kGemmBN / 2); c < (ch + 1) * (kGemmBN / 2); c += 16) {
                 float v[16];
                 tmem_ld16(taddr + c, v);
                 if (nsplit == 1) {
