@@ -1,7 +1,8 @@
 // Device helpers shared by the qgemm kernels (sm_100a only).
 //
 // Everything here is a thin wrapper over one PTX instruction (mbarrier, bulk
-// copy, mma.sync, fences) plus the bounded wait every pipeline uses: a wait on
+// and tensor copies, tcgen05, fences) plus the bounded wait every pipeline
+// uses: a wait on
 // an mbarrier gives up after about one second, records QGEMM_DEV_TIMEOUT in the
 // per-device error word and reports failure to the caller, which then unwinds
 // without issuing further work.
@@ -113,18 +114,11 @@ QG_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) 
         : "memory");
 }
 
-// Same, with an L2 eviction-priority hint (the weight stream is read once).
-QG_DEV void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
-                          uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
-        "%2, [%3], %4;" ::"r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
 // 2D tensor copy global -> this CTA's shared memory of the box at (x, y) of
-// the tensor map, completing on an mbarrier (same rules as below).
+// the tensor map (x in elements, a multiple of 16 bytes; y in rows),
+// completing on an mbarrier.  dst 128-byte aligned.  The whole box counts
+// toward the mbarrier's transaction bytes, out-of-range elements arriving as
+// zeros.
 QG_DEV void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -133,47 +127,12 @@ QG_DEV void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar
         : "memory");
 }
 
-// 2D tensor copy global -> this CTA's shared memory of the box at (x, y) of
-// the tensor map (x in elements, a multiple of 16 bytes; y in rows), with an
-// L2 cache policy.  dst 128-byte aligned.  The whole box counts toward the
-// mbarrier's transaction bytes, out-of-range elements arriving as zeros.
-QG_DEV void tma_load_2d_hint(void* dst, const void* tmap, int x, int y, uint64_t* bar, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
-        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
-QG_DEV uint64_t policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
 // --------------------------------------------------------- named barriers
 QG_DEV void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// ------------------------------------------------------------------ mma.sync
-// D = A(16x16, row) * B(16x8, col) + C, fp16 inputs, fp32 accumulate.
-QG_DEV void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                          uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
-// Same with C = 0 (starts a new accumulation).
-QG_DEV void mma_f16_16816_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
-}
 
 // --------------------------------------------------------------- tcgen05
 // Tensor memory (TMEM) and the 5th-generation tensor-core MMA.  Addresses are
@@ -192,7 +151,6 @@ QG_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {  // whole warp
 QG_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 QG_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 QG_DEV void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-QG_DEV void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 16 consecutive 32-bit columns: this thread's lane gets r[0..15].
 // No "memory" clobber: TMEM is ordered by tcgen05.wait::st/ld and the fences,
@@ -274,23 +232,8 @@ QG_DEV uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
     return d;
 }
 
-QG_DEV uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
 
-QG_DEV uint32_t hsub2_u32(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
 
-QG_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
 
 // byte permute with an immediate selector
 template <uint32_t SEL>

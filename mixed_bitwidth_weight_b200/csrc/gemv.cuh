@@ -440,7 +440,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
     // =================================================== producer warp
     if (warp == kGemvProducerWarp) {
         if (lane != 0) return;
-        const uint64_t policy = policy_evict_first();
         asm volatile("griddepcontrol.wait;" ::: "memory");  // activations come from xprep
         int pos = 0, pos_rel = 0;
         int64_t total = 0, total_rel = 0;
@@ -477,8 +476,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
             bulk_g2s(dst + 512, p.xcorr + (size_t)g * MP, (uint32_t)MP * 4, &s_full[slot]);
             const uint32_t* src = p.qw + (size_t)s_offs[j0] * p.N + (size_t)t * kGemvTileCols;
             for (int r = 0; r < wrows; ++r)
-                bulk_g2s_hint(dst + (size_t)(r + 1) * kGemvRowBytes, src + (size_t)r * p.N,
-                              (uint32_t)cols * 4, &s_full[slot], policy);
+                bulk_g2s(dst + (size_t)(r + 1) * kGemvRowBytes, src + (size_t)r * p.N, (uint32_t)cols * 4,
+                         &s_full[slot]);
             bulk_g2s(dst + (size_t)(1 + wrows) * kGemvRowBytes, p.xdec + (size_t)j0 * (REC / 2),
                      (uint32_t)nblk * REC, &s_full[slot]);
             if (++g == ng) { g = 0; ++t; }
