@@ -2,10 +2,9 @@
 //
 // Everything here is a thin wrapper over one PTX instruction (mbarrier, bulk
 // and tensor copies, tcgen05, fences) plus the bounded wait every pipeline
-// uses: a wait on
-// an mbarrier gives up after about one second, records QGEMM_DEV_TIMEOUT in the
-// per-device error word and reports failure to the caller, which then unwinds
-// without issuing further work.
+// uses: a wait on an mbarrier gives up after about one second, records
+// QGEMM_DEV_TIMEOUT in the per-device error word and reports failure to the
+// caller, which then unwinds without issuing further work.
 #pragma once
 
 #include <cuda_fp16.h>
