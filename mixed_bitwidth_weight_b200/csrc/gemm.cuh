@@ -93,61 +93,72 @@ QG_DEV int gemm_code_of_k(int b, int k) {
 }
 
 // x_p[m][k] = fp16(x[m][perm[k']] * 2^-shift[m]), k' = the code the B tile
-// holds at position k (gemm_code_of_k), one CTA per row, 8 k per
-// thread step (16-byte stores).  fp16 input: shift 0, a plain gather.  bf16
-// input: shift puts the row's largest magnitude in [2^14, 2^15), so the
-// conversion to fp16 is exact for every value within 2^24 of the maximum;
-// the GEMM multiplies the row of y by 2^shift.
+// holds at position k (gemm_code_of_k).  One CTA per kXpermRows rows (and
+// per k range when there are few rows): the permutation indices of a k chunk
+// are loaded once and serve every row, and the rows' gathers are issued
+// together.  fp16 input: shift 0, a plain
+// gather.  bf16 input: shift puts the row's largest magnitude in
+// [2^14, 2^15), so the conversion to fp16 is exact for every value within
+// 2^24 of the maximum; the GEMM multiplies the row of y by 2^shift.
+constexpr int kXpermRows = 8;  // one warp per row for the row maxima
+
 __global__ void __launch_bounds__(256) xperm_kernel(const XpermParams p) {
-    __shared__ int s_e[8];
-    const int64_t m = blockIdx.x;
-    const uint16_t* row = p.x + m * p.K;
-    int shift = 0;
-    if (p.x_bf16) {
+    __shared__ int s_shift[kXpermRows];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m0 = (int64_t)blockIdx.x * kXpermRows;
+    const int nrows = (int)min((int64_t)kXpermRows, (int64_t)p.M - m0);
+    if (threadIdx.x < kXpermRows) s_shift[threadIdx.x] = 0;
+    __syncthreads();
+    if (p.x_bf16 && warp < nrows) {
+        const uint16_t* row = p.x + (m0 + warp) * p.K;
         int e = 0;
-        for (int k = threadIdx.x; k < p.K; k += blockDim.x) e = max(e, (int)((row[k] >> 7) & 0xFF));
+#pragma unroll 8
+        for (int k = lane; k < p.K; k += 32) e = max(e, (int)((row[k] >> 7) & 0xFF));
 #pragma unroll
         for (int o = 16; o; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
-        if ((threadIdx.x & 31) == 0) s_e[threadIdx.x >> 5] = e;
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            int v = threadIdx.x < 8 ? s_e[threadIdx.x] : 0;
-#pragma unroll
-            for (int o = 4; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-            if (threadIdx.x == 0) s_e[0] = v;
+        const int shift = (e == 0) ? 0 : e - 141;  // max < 2^(E-126); 2^(E-127-shift) = 2^14
+        if (lane == 0) {
+            s_shift[warp] = shift;
+            if (blockIdx.y == 0) p.xshift[m0 + warp] = shift;
         }
-        __syncthreads();
-        shift = (s_e[0] == 0) ? 0 : s_e[0] - 141;  // max < 2^(E-126); 2^(E-127-shift) = 2^14
-        if (threadIdx.x == 0) p.xshift[m] = shift;
     }
-    const int s1 = shift / 2, s2 = shift - shift / 2;  // 2^-shift as two normal factors
-    const float f1 = __int_as_float((127 - s1) << 23), f2 = __int_as_float((127 - s2) << 23);
-    for (int k0 = threadIdx.x * 8; k0 < p.K; k0 += blockDim.x * 8) {
+    __syncthreads();
+    float f1[kXpermRows], f2[kXpermRows];  // 2^-shift as two normal factors
+#pragma unroll
+    for (int r = 0; r < kXpermRows; ++r) {
+        const int sh = s_shift[r], s1 = sh / 2, s2 = sh - sh / 2;
+        f1[r] = __int_as_float((127 - s1) << 23);
+        f2[r] = __int_as_float((127 - s2) << 23);
+    }
+    // k range of this CTA (gridDim.y splits k when there are few rows)
+    const int kchunk = ((p.K / 32 + gridDim.y - 1) / gridDim.y) * 32;
+    const int kx0 = blockIdx.y * kchunk, kx1 = min(p.K, kx0 + kchunk);
+    for (int k0 = kx0 + threadIdx.x * 8; k0 < kx1; k0 += blockDim.x * 8) {
         const int blk = k0 >> 5;
         const int b = p.bits[blk];  // the GEMM refuses a schedule with a bad width
         int idx[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) idx[u] = p.perm[blk * 32 + gemm_code_of_k(b, (k0 & 31) + u)];
-        uint32_t v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            uint16_t h[2];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const int a = idx[2 * u + t];
-                uint16_t raw = 0;
-                if ((unsigned)a < (unsigned)p.K) raw = row[a];
-                else set_dev_error(QGEMM_DEV_BAD_PERM);
-                if (p.x_bf16) {
-                    const float f = __uint_as_float((uint32_t)raw << 16) * f1 * f2;
-                    h[t] = __half_as_ushort(__float2half_rn(f));
-                } else {
-                    h[t] = raw;
-                }
+        for (int u = 0; u < 8; ++u) {
+            idx[u] = p.perm[blk * 32 + gemm_code_of_k(b, (k0 & 31) + u)];
+            if ((unsigned)idx[u] >= (unsigned)p.K) {
+                set_dev_error(QGEMM_DEV_BAD_PERM);
+                idx[u] = -1;
             }
-            v[u] = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
         }
-        *reinterpret_cast<uint4*>(p.xp + m * p.K + k0) = make_uint4(v[0], v[1], v[2], v[3]);
+#pragma unroll
+        for (int r = 0; r < kXpermRows; ++r) {
+            if (r >= nrows) break;
+            const uint16_t* row = p.x + (m0 + r) * p.K;
+            uint32_t h[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t raw = idx[u] >= 0 ? (uint32_t)row[idx[u]] : 0u;
+                h[u] = p.x_bf16 ? (uint32_t)__half_as_ushort(__float2half_rn(__uint_as_float(raw << 16) * f1[r] * f2[r]))
+                                : raw;
+            }
+            *reinterpret_cast<uint4*>(p.xp + (m0 + r) * p.K + k0) =
+                make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+        }
     }
 }
 

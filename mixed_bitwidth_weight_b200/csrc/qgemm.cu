@@ -491,7 +491,13 @@ int run_gemm(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     xq.M = M;
     xq.K = K;
     xq.x_bf16 = bf16;
-    xperm_kernel<<<(unsigned)M, 256, 0, stream>>>(xq);
+    {
+        // rows in groups of kXpermRows; split k so that there are about 4
+        // CTAs per SM, each with at least 2048 k
+        const int64_t rg = (M + kXpermRows - 1) / kXpermRows;
+        const int64_t kspl = std::max<int64_t>(1, std::min<int64_t>(K / 2048, (4 * dev->sms + rg - 1) / rg));
+        xperm_kernel<<<dim3((unsigned)rg, (unsigned)kspl), 256, 0, stream>>>(xq);
+    }
     if ((st = launch_status()) != QGEMM_OK) return st;
 
     GemmParams p;
