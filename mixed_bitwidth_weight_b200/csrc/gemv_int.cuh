@@ -20,14 +20,15 @@
 //   -z * sum(x_int); each group's integer sum is then converted once and
 //   multiplied by the (group, column) scale and 2^-e in fp32.
 //
-// Work split as in gemv.cuh: units (256-column tile, 128-row group) split by
-// packed-word cost into one range per CTA (two CTAs per SM for M <= 2, one
-// for M <= 4).  Three lanes of warp 8 stream each unit into a shared-memory
-// ring of 1 KB rows: its word rows (2D tensor copies of 2^i rows x 256
-// columns, one per set bit of the row count, so a unit takes two or three
-// copies instead of one per row), its scale row (a bulk copy) and its
-// activation records (a bulk copy).  Weights go out before the wait for the activation kernel;
-// records after it.  Consumer warps 0-7: warp w decodes block w/2 of the unit
+// Work split as in gemv.cuh, with units of (256-column tile, two 128-row
+// groups) = 8 blocks: the units of all tiles are cut into one contiguous range
+// per CTA (two CTAs per SM for M <= 2, one for M <= 4) of equal cost (word
+// rows plus one per unit).  Two copy warps stream each unit into a
+// shared-memory ring of 1 KB rows: its word rows (2D tensor copies of 2^i rows
+// x 256 columns, one per set bit of the row count), its scale rows (bulk
+// copies) and its activation records (a bulk copy, from a warp of its own:
+// weights are issued before the wait for the activation kernel, records after
+// it).  Consumer warps 0-7: warp w decodes block w/2 of each group of the unit
 // for the 128 columns of half w%2, four adjacent columns per thread (one
 // 16-byte load per word row); the four block slots are added in shared memory
 // when a tile is done.  A tile shared with other CTAs leaves a partial sum in
@@ -43,7 +44,7 @@
 namespace qg {
 
 constexpr int kIntMaxM = 4;
-constexpr int kIntThreads = kGemvDecThreads + 32;
+constexpr int kIntThreads = kGemvDecThreads + 64;  // 8 consumer warps, 2 copy warps
 constexpr int kIntRowBytes = 1024;   // one ring row: 256 words (a box row lands densely)
 constexpr int kIntBoxMaps = 7;       // tensor maps with box heights 1, 2, 4, ..., 64 rows
 constexpr int kIntUnitGroups = 2;    // 128-row groups per unit
@@ -363,21 +364,25 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
         return int_unit_rows(s_offs[bb] - s_offs[a], bb - a, REC);
     };
 
-    // =================================================== producer warp
-    // Lanes 0, 1 and 2 split each unit's copies: word rows (2D boxes), the
-    // scale row, the activation records.  One copy instruction takes a fixed
-    // issue time whatever its size, so three issuers keep the ring fuller.
-    // The three lanes take the same ring positions and the same waits, in the
-    // same order, and agree on every wait's outcome, so they issue the same
-    // units.
-    if (warp == kGemvDecWarps) {
-        if (lane > 2) return;
+    // =================================================== producer warps
+    // Three issuers split each unit's copies: lane 0 of warp 8 the word rows
+    // (2D boxes), lane 1 of warp 8 the scale rows, lane 0 of warp 9 the
+    // activation records.  A copy instruction can wait for room in the SM's
+    // copy queue, so the records, which the activation kernel may only just
+    // have written, get a warp of their own and are not held behind the
+    // weights that the other lanes issue ahead of them.  Every issuer takes the
+    // same ring positions and the same waits, in the same order, so they issue
+    // the same units; lanes 0 and 1 of warp 8 agree on every wait's outcome.
+    if (warp >= kGemvDecWarps) {
+        const int role = (warp == kGemvDecWarps) ? (lane < 2 ? lane : 3) : (lane == 0 ? 2 : 3);
+        if (role > 2) return;
+        const unsigned peers = (role == 2) ? 0x1u : 0x3u;
         auto issue = [&](int k, int t, int g, int row) {
             const int j0 = g * kIntUnitBlocks, j1 = min(j0 + kIntUnitBlocks, nb);
             const int r0 = s_offs[j0], wrows = s_offs[j1] - r0;
             uint64_t* bar = &s_full[k & (kGemvSlots - 1)];
             uint8_t* dst = s_ring + (size_t)row * kIntRowBytes;
-            if (lane == 0) {
+            if (role == 0) {
                 mbar_arrive_expect_tx(bar, (uint32_t)(wrows * kIntRowBytes));
                 int r = 0;
 #pragma unroll 1
@@ -387,7 +392,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                                     bar);
                         r += 1 << i;
                     }
-            } else if (lane == 1) {
+            } else if (role == 1) {
                 const int cols = min(kGemvTileCols, p.N - t * kGemvTileCols);
                 const int g0 = g * kIntUnitGroups, ngr = min(kIntUnitGroups, ng - g0);
                 mbar_arrive_expect_tx(bar, (uint32_t)(ngr * cols * 2));
@@ -401,8 +406,8 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                          bar);
             }
         };
-        // Units that fit the ring and the slots before any release: weights
-        // and scales first, then (once the activation kernel is done) records.
+        // Units that fit the ring and the slots before any release; the
+        // records issuer first waits for the activation kernel.
         int npre = 0;
         {
             int pp = 0, gg = gf;
@@ -418,22 +423,13 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                 if (++gg == nu) gg = 0;
             }
         }
+        if (role == 2) asm volatile("griddepcontrol.wait;" ::: "memory");  // records come from xprep_int
         int pos = 0;
         int64_t total = 0;
         int t = t0, g = gf;
         for (int k = 0; k < npre; ++k) {
-            const int row = ring_alloc(pos, total, rows_of(g), R);
-            if (lane != 2) issue(k, t, g, row);
+            issue(k, t, g, ring_alloc(pos, total, rows_of(g), R));
             if (++g == nu) { g = 0; ++t; }
-        }
-        if (lane == 2) {
-            asm volatile("griddepcontrol.wait;" ::: "memory");  // activation records come from xprep_int
-            int pp = 0, tt = t0, gg = gf;
-            int64_t tot = 0;
-            for (int k = 0; k < npre; ++k) {
-                issue(k, tt, gg, ring_alloc(pp, tot, rows_of(gg), R));
-                if (++gg == nu) { gg = 0; ++tt; }
-            }
         }
         int pos_rel = 0;
         int64_t total_rel = 0;
@@ -451,7 +447,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
             // rows exceed R
             while (k - k_rel >= kGemvSlots || (ptotal - total_rel > R && k_rel < k)) {
                 const bool w = mbar_wait(&s_empty[k_rel & (kGemvSlots - 1)], (uint32_t)((k_rel / kGemvSlots) & 1));
-                if (!__all_sync(0x7u, w)) {
+                if (!__all_sync(peers, w)) {
                     ok = false;
                     break;
                 }
@@ -464,9 +460,10 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
             if (++g == nu) { g = 0; ++t; }
         }
         if (!ok) {
+            // let this issuer's copies in flight land before the CTA can exit
             s_misc[3] = 1;
             for (int kk = k_rel; kk < k; ++kk)
-                mbar_wait(&s_full[kk & (kGemvSlots - 1)], (uint32_t)((kk / kGemvSlots) & 1));
+                if (!mbar_wait(&s_full[kk & (kGemvSlots - 1)], (uint32_t)((kk / kGemvSlots) & 1))) break;
         }
         return;
     }
