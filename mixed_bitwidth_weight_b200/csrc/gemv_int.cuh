@@ -333,7 +333,7 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
     if (bad) atomicOr(&s_misc[0], 1);
     if (tid == 0) {
         for (int i = 0; i < kGemvSlots; ++i) {
-            mbar_init(&s_full[i], 3);  // the three issuing lanes of the producer warp
+            mbar_init(&s_full[i], 3);  // the three issuers of the copy warps
             mbar_init(&s_empty[i], kGemvDecWarps);
         }
         fence_mbar_init();
