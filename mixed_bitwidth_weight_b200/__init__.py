@@ -94,6 +94,49 @@ def _dev(t, dtype, name):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _shape_error(msg):
+    raise ValueError(msg)
+
+
+def _check_schedule_tensors(K, bits, offs):
+    if K % 32 != 0:
+        _shape_error(f"K = {K} is not a multiple of 32")
+    if bits.numel() != K // 32:
+        _shape_error(f"bits has {bits.numel()} entries, K/32 = {K // 32} expected")
+    if offs.numel() != K // 32 + 1:
+        _shape_error(f"offs has {offs.numel()} entries, K/32 + 1 = {K // 32 + 1} expected")
+
+
+def _check_qgemm_shapes(x, perm, qw, scales, bits, offs, y):
+    """Shapes of one qgemm call, checked before any pointer reaches the C ABI
+    (a mismatch there would read or write past the end of a tensor)."""
+    if x.dim() != 2 or y.dim() != 2:
+        _shape_error("x and y must be 2-D ([M, K] and [M, N])")
+    M, K = x.shape
+    if y.shape[0] != M:
+        _shape_error(f"y has {y.shape[0]} rows, x has {M}")
+    N = y.shape[1]
+    if perm.numel() != K:
+        _shape_error(f"perm has {perm.numel()} entries, K = {K} expected")
+    if qw.dim() != 2 or qw.shape[1] != N:
+        _shape_error(f"qw must be [qw_rows, N = {N}], got {tuple(qw.shape)}")
+    G = (K + 127) // 128
+    if scales.numel() != G * N or (scales.dim() == 2 and tuple(scales.shape) != (G, N)):
+        _shape_error(f"scales must be [ceil(K/128) = {G}, N = {N}], got {tuple(scales.shape)}")
+    _check_schedule_tensors(K, bits, offs)
+
+
+def _check_same_device(*tensors):
+    """Every tensor on the current CUDA device (the call runs on its stream)."""
+    import torch
+    if not any(t.is_cuda for t in tensors):
+        return  # host tensors: refused by the pointer checks that follow
+    cur = torch.cuda.current_device()
+    for t in tensors:
+        if t.is_cuda and t.device.index != cur:
+            raise ValueError(f"tensor on cuda:{t.device.index}, but the current device is cuda:{cur}")
+
+
 def _host_u8(a):
     return np.ascontiguousarray(np.asarray(a), dtype=np.uint8)
 
@@ -149,8 +192,14 @@ def qgemm_device_error(clear: bool = True) -> int:
 def qgemm_pack(codes, bits, offs, qw, stream=None):
     """codes uint8 [K, N] -> qw int32/uint32 [qw_rows, N] (all CUDA tensors)."""
     import torch
+    if codes.dim() != 2 or qw.dim() != 2:
+        _shape_error("codes and qw must be 2-D ([K, N] and [qw_rows, N])")
     K, N = codes.shape
     rows = qw.shape[0]
+    if qw.shape[1] != N:
+        _shape_error(f"qw has {qw.shape[1]} columns, codes has {N}")
+    _check_schedule_tensors(K, bits, offs)
+    _check_same_device(codes, bits, offs, qw)
     _ok(_lib.qgemm_pack(_dev(codes, torch.uint8, "codes"), _dev(bits, torch.uint8, "bits"),
                         _dev(offs, torch.int32, "offs"), K, N, rows,
                         _dev(qw, (torch.int32, torch.uint32), "qw"), _stream(stream)), "qgemm_pack")
@@ -160,7 +209,16 @@ def qgemm_pack(codes, bits, offs, qw, stream=None):
 def qgemm_dequant(qw, scales, bits, offs, w, stream=None):
     """qw [qw_rows, N], scales fp16 [ceil(K/128), N] -> w fp16 [K, N]."""
     import torch
+    if w.dim() != 2 or qw.dim() != 2:
+        _shape_error("w and qw must be 2-D ([K, N] and [qw_rows, N])")
     K, N = w.shape
+    if qw.shape[1] != N:
+        _shape_error(f"qw has {qw.shape[1]} columns, w has {N}")
+    G = (K + 127) // 128
+    if scales.numel() != G * N or (scales.dim() == 2 and tuple(scales.shape) != (G, N)):
+        _shape_error(f"scales must be [ceil(K/128) = {G}, N = {N}], got {tuple(scales.shape)}")
+    _check_schedule_tensors(K, bits, offs)
+    _check_same_device(qw, scales, bits, offs, w)
     _ok(_lib.qgemm_dequant(_dev(qw, (torch.int32, torch.uint32), "qw"), qw.shape[0],
                            _dev(scales, torch.float16, "scales"), _dev(bits, torch.uint8, "bits"),
                            _dev(offs, torch.int32, "offs"), K, N, _dev(w, torch.float16, "w"),
@@ -171,6 +229,8 @@ def qgemm_dequant(qw, scales, bits, offs, w, stream=None):
 def qgemm(x, perm, qw, scales, bits, offs, y, ws=None, stream=None):
     """y [M, N] fp16 = x[:, perm] . dequant(qw); x fp16 or bf16 [M, K]."""
     import torch
+    _check_qgemm_shapes(x, perm, qw, scales, bits, offs, y)
+    _check_same_device(x, perm, qw, scales, bits, offs, y, *(() if ws is None else (ws,)))
     M, K = x.shape
     N = y.shape[1]
     if x.dtype == torch.float16:
@@ -200,6 +260,8 @@ def qgemm_decode_noalloc(x, perm, qw, scales, bits, offs, y, stream=None):
     allocate device memory).  Calls that overlap on the GPU race on that
     buffer; the first call on a device should come before any stream capture."""
     import torch
+    _check_qgemm_shapes(x, perm, qw, scales, bits, offs, y)
+    _check_same_device(x, perm, qw, scales, bits, offs, y)
     M, K = x.shape
     N = y.shape[1]
     if x.dtype == torch.float16:

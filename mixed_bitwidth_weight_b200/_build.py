@@ -36,7 +36,10 @@ def _sources():
 
 
 def _digest() -> str:
-    h = hashlib.sha1(" ".join(FLAGS).encode())
+    """Hash of the sources and the flags, independent of where the tree lives
+    (flags are hashed with the tree's root replaced by a placeholder), so the
+    same sources give the same digest on every machine."""
+    h = hashlib.sha1(" ".join(f.replace(ROOT, "<root>") for f in FLAGS).encode())
     for f in _sources():
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())

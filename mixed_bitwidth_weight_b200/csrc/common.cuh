@@ -31,6 +31,9 @@ __device__ int g_dev_error = 0;
 
 QG_DEV void set_dev_error(int code) { atomicOr(&g_dev_error, code); }
 
+// Block widths the format allows: {2, 3, 4, 5, 6, 8}.
+QG_DEV bool width_ok(int b) { return b == 2 || b == 3 || b == 4 || b == 5 || b == 6 || b == 8; }
+
 QG_DEV uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -10,7 +10,6 @@
 
 namespace qg {
 
-QG_DEV bool width_ok(int b) { return b == 2 || b == 3 || b == 4 || b == 5 || b == 6 || b == 8; }
 
 // Local consistency of block j of the schedule.  Checking this for every
 // block a kernel touches keeps all of its word-row accesses inside

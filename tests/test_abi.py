@@ -142,3 +142,58 @@ def test_gemm_plan_and_workspace():
     ks = big["ring"]
     assert ks == 4 and big["grid"] == ks
     assert q.qgemm_workspace_bytes(17, 65536, 8) >= 17 * 65536 * 2 + ks * 256 * 256 * 4
+
+
+def _cpu_args(M=2, K=256, N=64):
+    import torch
+    nb = K // 32
+    rows = 2 * nb
+    return dict(
+        x=torch.zeros(M, K, dtype=torch.float16), perm=torch.arange(K, dtype=torch.int32),
+        qw=torch.zeros(rows, N, dtype=torch.int32),
+        scales=torch.zeros((K + 127) // 128, N, dtype=torch.float16),
+        bits=torch.full((nb,), 2, dtype=torch.uint8),
+        offs=torch.arange(0, 2 * nb + 1, 2, dtype=torch.int32),
+        y=torch.zeros(M, N, dtype=torch.float16))
+
+
+@pytest.mark.parametrize("fn", ["qgemm", "qgemm_decode_noalloc"])
+@pytest.mark.parametrize("bad", ["y_rows", "perm", "qw_cols", "scales", "bits", "offs", "x_1d"])
+def test_binding_rejects_mismatched_shapes(fn, bad):
+    """The binding checks every shape before a pointer reaches the C ABI, so a
+    mismatch is a ValueError on the host, never an out-of-bounds access."""
+    import torch
+    a = _cpu_args()
+    if bad == "y_rows":
+        a["y"] = torch.zeros(4, 64, dtype=torch.float16)
+    elif bad == "perm":
+        a["perm"] = torch.arange(255, dtype=torch.int32)
+    elif bad == "qw_cols":
+        a["qw"] = torch.zeros(16, 72, dtype=torch.int32)
+    elif bad == "scales":
+        a["scales"] = torch.zeros(3, 64, dtype=torch.float16)
+    elif bad == "bits":
+        a["bits"] = torch.full((7,), 2, dtype=torch.uint8)
+    elif bad == "offs":
+        a["offs"] = torch.zeros(8, dtype=torch.int32)
+    elif bad == "x_1d":
+        a["x"] = torch.zeros(256, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        getattr(q, fn)(**a)
+
+
+def test_binding_shapes_ok_then_needs_cuda_tensors():
+    """Consistent shapes pass the shape checks; host tensors are then refused."""
+    with pytest.raises(TypeError):
+        q.qgemm(**_cpu_args())
+
+
+def test_pack_and_dequant_reject_mismatched_shapes():
+    import torch
+    a = _cpu_args()
+    with pytest.raises(ValueError):
+        q.qgemm_pack(torch.zeros(256, 64, dtype=torch.uint8), a["bits"], a["offs"],
+                     torch.zeros(16, 56, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        q.qgemm_dequant(a["qw"], torch.zeros(3, 64, dtype=torch.float16), a["bits"], a["offs"],
+                        torch.zeros(256, 64, dtype=torch.float16))
