@@ -192,7 +192,7 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
  *     that overlap on the GPU (other streams, other threads) race on the
  *     buffer and give wrong results: order them, e.g. on one stream.
  *   Returns a qgemm_status as qgemm(). */
-#define QGEMM_NOALLOC_SCRATCH_BYTES ((size_t)6 << 20)
+#define QGEMM_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 
 int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm,
                          const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scales,

@@ -251,7 +251,7 @@ def qgemm(x, perm, qw, scales, bits, offs, y, ws=None, stream=None):
     return y
 
 
-NOALLOC_SCRATCH_BYTES = 6 << 20
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def qgemm_decode_noalloc(x, perm, qw, scales, bits, offs, y, stream=None):

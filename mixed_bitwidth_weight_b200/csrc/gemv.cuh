@@ -7,16 +7,17 @@
 //
 // 1. xprep_kernel gathers the activations once through perm, in the order the
 //    decoder emits codes (code_of_k), pre-scaled by 2^-P, laid out as the
-//    tensor core's B operand, and computes a per-(group, token) correction.
+//    tensor core's B operand.
 // 2. gemv_kernel, launched as a programmatic dependent of xprep_kernel: it
 //    starts setting up at once and waits for xprep only before it copies data.
 //
 // Decode without a conversion step.  A code q at mantissa bits [P, P+b) of a
 // 16-bit half ORed with 0x6400 is the fp16 number h = 1024 + q * 2^P (one
-// lop3 or prmt per two codes).  With x' = x * 2^-P as the other operand,
-// sum x' h = sum x (q - z) + sum x' (1024 + z 2^P); the second sum is the
-// correction, known before the weights arrive, subtracted once per group in
-// fp32.  Both operands are exact fp16 values.
+// lop3 or prmt per two codes); one fp16x2 subtraction of 1024 + z 2^P, exact,
+// leaves (q - z) 2^P.  With x' = x * 2^-P as the other operand every product
+// is x (q - z) exactly, so the group sum needs no correction term: an
+// activation outlier over a weight row at its zero point adds exactly zero,
+// and nothing large is subtracted after the accumulation.
 //
 // Tensor cores.  Each decoder thread owns one output column (one TMEM lane)
 // and writes the decoded codes of its column straight into tensor memory with
@@ -24,7 +25,7 @@
 // N = 16 tokens, K = 16) with A read from TMEM and B = the staged activations
 // in shared memory, accumulating one 128-row group in fp32 in TMEM.  The
 // decoder threads then read their column's group sum back (tcgen05.ld),
-// subtract the correction and apply the (group, column) scale.  The legacy
+// and apply the (group, column) scale.  The legacy
 // warp-level mma.sync path is not used: on sm_100 it costs about a dozen
 // instructions per MMA, which made decode issue-bound.
 //
@@ -39,7 +40,7 @@
 //
 // Roles.  Warps 0-7: decoders and epilogue, thread t = column t of the tile
 // (TMEM lane t % 128 of subtile t / 128).  Warp 8: producer, one lane copies
-// each unit's scale row, correction, word rows and activation records with
+// each unit's scale row, word rows and activation records with
 // cp.async.bulk into a ring of shared-memory rows.  Warp 9: TMEM allocation
 // and, on one lane, the MMA issue.
 #pragma once
@@ -65,7 +66,6 @@ constexpr int kGemvDCol = kGemvAStages * 128;           // first TMEM column of 
 
 struct GemvParams {
     const __half* xdec;    // [nb][4][MP][8] activations in decoder order, scaled by 2^-P
-    const float* xcorr;    // [ng][MP] correction per (group, token)
     const int* xshift;     // [16] per-row power-of-two scale of bf16 input (0 for fp16)
     const uint32_t* qw;
     int64_t qw_rows;
@@ -85,7 +85,6 @@ struct XprepParams {
     const uint8_t* bits;
     const int32_t* offs;
     __half* xdec;
-    float* xcorr;
     int* xshift;
     int M, K, nb, mp, x_bf16;
 };
@@ -101,22 +100,34 @@ QG_DEV int code_of_k(int b, int k) {
         default: return 8 * (j >> 2) + (j & 3) + 4 * h;  // 3, 5, 6
     }
 }
-QG_DEV int shift_of_k(int b, int k) {
-    const int j = k >> 1;
-    switch (b) {
-        case 2: return 2 * (j & 3);
-        case 3: return ((j & 3) == 1) ? 3 : ((j & 3) == 2) ? 6 : 0;
-        case 4: return (j & 1) ? 4 : 0;
-        case 5: return (j & 1) ? 5 : 0;
-        default: return 0;  // 6, 8
-    }
+
+// Mantissa bit P of the codes in fp16x2 value j of a block (both halves).
+__host__ __device__ constexpr int shift_of_pair(int b, int j) {
+    return b == 2 ? 2 * (j & 3)
+         : b == 3 ? (((j & 3) == 1) ? 3 : ((j & 3) == 2) ? 6 : 0)
+         : b == 4 ? ((j & 1) ? 4 : 0)
+         : b == 5 ? ((j & 1) ? 5 : 0)
+         : 0;  // 6, 8
+}
+QG_DEV int shift_of_k(int b, int k) { return shift_of_pair(b, k >> 1); }
+
+// fp16x2 bits of 1024 + z * 2^P in both halves, z = 2^(b-1): the bias that
+// fp16x2 value j of a block carries.
+__host__ __device__ constexpr uint32_t bias_of_pair(int b, int j) {
+    return (0x6400u | (1u << (b - 1 + shift_of_pair(b, j)))) * 0x10001u;
+}
+
+QG_DEV uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 // The 32 codes of one block in one column as 16 fp16x2 values
 // h = 1024 + q * 2^P, in the order code_of_k describes.  w points at word 0
 // of the block in this column; word i is at w + i * kGemvRowBytes.
 template <int B>
-QG_DEV void decode_block(const uint8_t* w, uint32_t (&P)[16]) {
+QG_DEV void decode_block_biased(const uint8_t* w, uint32_t (&P)[16]) {
     auto word = [&](int i) { return *reinterpret_cast<const uint32_t*>(w + i * kGemvRowBytes); };
     if constexpr (B == 2) {
 #pragma unroll
@@ -188,6 +199,16 @@ QG_DEV void decode_block(const uint8_t* w, uint32_t (&P)[16]) {
     }
 }
 
+// The 32 codes of one block in one column as 16 fp16x2 values
+// (q - z) * 2^P, in the order code_of_k describes.  w points at word 0 of the
+// block in this column; word i is at w + i * kGemvRowBytes.
+template <int B>
+QG_DEV void decode_block(const uint8_t* w, uint32_t (&P)[16]) {
+    decode_block_biased<B>(w, P);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) P[j] = hsub2_u32(P[j], bias_of_pair(B, j));  // exact
+}
+
 // A full group of 4 blocks of width B: decode each block of this thread's
 // column and store it to the TMEM A stage (16 columns per block).  w0 = the
 // group's first word row at this column.
@@ -254,7 +275,7 @@ QG_DEV int ring_alloc(int& pos, int64_t& total, int need, int R) {
 }
 
 // Ring rows of a unit with `wrows` word rows and `nblk` blocks: the scale row
-// (which also holds the correction at byte 512), the word rows, then the
+// (its first 512 bytes hold the scales), the word rows, then the
 // activation records (64 * MP bytes per block).
 QG_DEV int unit_rows(int wrows, int nblk, int mp) {
     return 1 + wrows + (nblk * 64 * mp + kGemvRowBytes - 1) / kGemvRowBytes;
@@ -264,13 +285,11 @@ QG_DEV int unit_rows(int wrows, int nblk, int mp) {
 // One warp per block: lane k = position in the decoder's order.  Writes the
 // activation of every token (scaled by 2^-P) into the block's record
 // [4 k-chunks][MP tokens][8], the B-operand layout of the MMA (tokens >= M
-// are zeros), and reduces the correction sum x' * (1024 + z * 2^P) per
-// 128-row group (8 warps = 2 groups per CTA).  bf16 input is first scaled per
+// are zeros).  bf16 input is first scaled per
 // row by 2^-shift so that the row's largest magnitude lands in [2^14, 2^15).
 __global__ void __launch_bounds__(256) xprep_kernel(const XprepParams p) {
     asm volatile("griddepcontrol.launch_dependents;");
     __shared__ int s_shift[16];
-    __shared__ float s_bc[8][16];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x < 16) s_shift[threadIdx.x] = 0;
     __syncthreads();
@@ -305,11 +324,9 @@ __global__ void __launch_bounds__(256) xprep_kernel(const XprepParams p) {
             src = 0;
         }
     }
-    const float offset = (float)(1024 + (1 << (b - 1)) * (1 << P));
     const float inv2p = __int_as_float((127 - P) << 23);
     __half* rec = p.xdec + (size_t)j * 4 * p.mp * 8;
     for (int m = 0; m < p.mp; ++m) {
-        float corr = 0.f;
         __half xs = __float2half_rn(0.f);
         if (live && m < p.M) {
             const uint16_t raw = reinterpret_cast<const uint16_t*>(p.x)[(size_t)m * p.K + src];
@@ -322,21 +339,8 @@ __global__ void __launch_bounds__(256) xprep_kernel(const XprepParams p) {
                 v = __half2float(__ushort_as_half(raw));
             }
             xs = __float2half_rn(v * inv2p);  // exact unless below fp16 normals
-            corr = __half2float(xs) * offset;
         }
         if (live) rec[((lane >> 3) * p.mp + m) * 8 + (lane & 7)] = xs;
-#pragma unroll
-        for (int o = 16; o; o >>= 1) corr += __shfl_xor_sync(0xffffffffu, corr, o);
-        if (lane == 0) s_bc[warp][m] = corr;
-    }
-    __syncthreads();
-    // group gl of this CTA = blocks 4gl..4gl+3 = warps 4gl..4gl+3
-    if (threadIdx.x < 2 * p.mp) {
-        const int gl = threadIdx.x / p.mp, m = threadIdx.x - gl * p.mp;
-        const int gg = blockIdx.x * 2 + gl;
-        if (gg * kGemvGroupBlocks < p.nb)
-            p.xcorr[(size_t)gg * p.mp + m] = s_bc[4 * gl][m] + s_bc[4 * gl + 1][m] +
-                                              s_bc[4 * gl + 2][m] + s_bc[4 * gl + 3][m];
     }
 }
 
@@ -469,11 +473,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
             const int row = ring_alloc(pos, total, need, R);
             const int slot = k & (kGemvSlots - 1);
             const int cols = min(kGemvTileCols, p.N - t * kGemvTileCols);
-            mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cols * 2 + MP * 4 + wrows * cols * 4 + nblk * REC));
+            mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cols * 2 + wrows * cols * 4 + nblk * REC));
             uint8_t* dst = s_ring + (size_t)row * kGemvRowBytes;
             bulk_g2s(dst, p.scales + (size_t)g * p.N + (size_t)t * kGemvTileCols, (uint32_t)cols * 2,
                      &s_full[slot]);
-            bulk_g2s(dst + 512, p.xcorr + (size_t)g * MP, (uint32_t)MP * 4, &s_full[slot]);
             const uint32_t* src = p.qw + (size_t)s_offs[j0] * p.N + (size_t)t * kGemvTileCols;
             for (int r = 0; r < wrows; ++r)
                 bulk_g2s(dst + (size_t)(r + 1) * kGemvRowBytes, src + (size_t)r * p.N, (uint32_t)cols * 4,
@@ -613,10 +616,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         named_bar_sync(1, kGemvDecThreads);
     };
 
-    // epilogue of unit k: group sum from TMEM, minus the correction, times the scale
-    float prev_sc = 0.f, prev_corr[MP];
-#pragma unroll
-    for (int i = 0; i < MP; ++i) prev_corr[i] = 0.f;
+    // epilogue of unit k: group sum from TMEM times the scale
+    float prev_sc = 0.f;
     auto epilogue = [&](int k) {
         const int buf = k & 1;
         if (!aborted && !s_misc[2] && mbar_wait(&s_dfull[buf], (uint32_t)((k >> 1) & 1))) {
@@ -628,7 +629,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_dempty[buf]);
 #pragma unroll
-            for (int tok = 0; tok < MP; ++tok) acc[tok] += prev_sc * (d[tok] - prev_corr[tok]);
+            for (int tok = 0; tok < MP; ++tok) acc[tok] = fmaf(prev_sc, d[tok], acc[tok]);
         } else {
             aborted = true;
             s_misc[2] = 1;
@@ -646,9 +647,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         const int row = ring_alloc(pos, total, unit_rows(s_offs[j1] - o0, nblk, MP), R);
         const int slot = k & (kGemvSlots - 1);
         const int s = k % kGemvAStages;
-        float sc = 0.f, corr[MP];
-#pragma unroll
-        for (int i = 0; i < MP; ++i) corr[i] = 0.f;
+        float sc = 0.f;
         if (!aborted && (s_misc[2] || !mbar_wait(&s_full[slot], (uint32_t)((k / kGemvSlots) & 1)))) {
             aborted = true;
             s_misc[2] = 1;
@@ -666,8 +665,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
         if (!aborted) {
             const uint8_t* ub = s_ring + (size_t)row * kGemvRowBytes;
             sc = __half2float(reinterpret_cast<const __half*>(ub)[ctid]);
-#pragma unroll
-            for (int i = 0; i < MP; ++i) corr[i] = reinterpret_cast<const float*>(ub + 512)[i];
             const uint8_t* wcol = ub + kGemvRowBytes + ctid * 4;
             const uint32_t ta = tmem + tlane + s * 128 + sub * 64;
             const int b0 = s_offs[j0 + 1] - o0;
@@ -718,8 +715,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
             }
         }
         prev_sc = sc;
-#pragma unroll
-        for (int i = 0; i < MP; ++i) prev_corr[i] = corr[i];
         if (++g == ng) { g = 0; ++t; }
     }
     epilogue(nunits - 1);

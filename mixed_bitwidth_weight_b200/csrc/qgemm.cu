@@ -3,14 +3,13 @@
 // This file is the library's only translation unit: it includes the kernels,
 // validates every argument on the host before anything is launched, sizes the
 // launches for the current device and maps CUDA failures to qgemm_status.
-#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 
 #include "common.cuh"
 #include "gemv.cuh"
-#include "gemv_i8.cuh"
+#include "gemv_int.cuh"
 #include "gemm.cuh"
 
 namespace {
@@ -22,7 +21,7 @@ constexpr int kVersion = 100;  // 0.1.0
 struct DeviceInfo {
     int sms = 0;
     bool gemv_attr[2] = {false, false};
-    bool i8_attr[3] = {false, false, false};
+    bool int_attr[3] = {false, false, false};
     bool gemm_attr[2] = {false, false};
 };
 
@@ -80,9 +79,9 @@ int64_t gemv_max_grid(int K, int N, int sms) {
     return std::min<int64_t>(U, (int64_t)4 * sms);
 }
 
-// Workspace: [tickets][partial slots][activation records][corrections][row shifts].
+// Workspace: [tickets][partial slots][activation records][row shifts].
 struct GemvWs {
-    size_t tickets, slots, xdec, xcorr, xshift, total;
+    size_t tickets, slots, xdec, xshift, total;
 };
 
 GemvWs gemv_ws_layout(int M, int K, int N, int sms) {
@@ -92,8 +91,7 @@ GemvWs gemv_ws_layout(int M, int K, int N, int sms) {
     w.tickets = 0;
     w.slots = align_up((size_t)gemv_tiles(N) * 4, 256);
     w.xdec = w.slots + align_up((size_t)gemv_max_grid(K, N, sms) * 2 * mp * kGemvTileCols * 4, 256);
-    w.xcorr = w.xdec + align_up((size_t)(nb + 8) * 64 * mp, 256);
-    w.xshift = w.xcorr + align_up((size_t)(gemv_groups(K) + 2) * mp * 4, 256);
+    w.xshift = w.xdec + align_up((size_t)(nb + 8) * 64 * mp, 256);
     w.total = w.xshift + 256;
     return w;
 }
@@ -148,7 +146,6 @@ int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     xp.bits = bits;
     xp.offs = offs;
     xp.xdec = reinterpret_cast<__half*>(w8 + L.xdec);
-    xp.xcorr = reinterpret_cast<float*>(w8 + L.xcorr);
     xp.xshift = reinterpret_cast<int*>(w8 + L.xshift);
     xp.M = M;
     xp.K = K;
@@ -160,7 +157,6 @@ int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
 
     GemvParams p;
     p.xdec = xp.xdec;
-    p.xcorr = xp.xcorr;
     p.xshift = xp.xshift;
     p.qw = qw;
     p.qw_rows = qw_rows;
@@ -199,15 +195,22 @@ int run_gemv(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
     return launch_status();
 }
 
-// ------------------------------------------- integer tensor-core GEMV
+// ----------------------------------------------------------- integer GEMV
 constexpr int kPathGemvInt = 0, kPathGemvTc = 1, kPathGemm = 2;
-// M served by the integer tensor-core GEMV (four tokens fill the MMA's
-// sixteen digit columns)
-constexpr int kIntPathMaxM = kI8MaxM;
+// M served by the integer GEMV (measured: above four tokens the tensor-core
+// GEMV is faster)
+constexpr int kIntPathMaxM = 4;
 // M served by the allocation-free decode entry point
-constexpr int kNoAllocMaxM = kI8MaxM;
+constexpr int kNoAllocMaxM = 4;
 
-int i8_mp(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
+int int_mp(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
+int int_ctas_per_sm(int mp) { return mp <= 2 ? 2 : 1; }
+
+size_t int_fixed_smem(int nb, int mp) {
+    const size_t o = align_up((size_t)(nb + 1) * 4, 16) + 2 * kGemvSlots * 8 + 64 +
+                     (size_t)3 * kGemvTileCols * mp * 4;
+    return align_up(o, 1024);
+}
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime
 // (the library does not link the driver library itself).
@@ -229,177 +232,79 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// Tensor maps of a decode call depend only on the weight and scale pointers
-// and their shapes, so they are encoded once and cached: an eager decode loop
-// then spends no host time on them.  The cache is keyed by (device, pointer,
-// rows, columns) and replaced round-robin.
-struct I8MapCacheEntry {
-    int dev;
-    const void* qw;
-    const void* sc;
-    int64_t rows;
-    int n, g;
-    I8Maps maps;
-};
-constexpr int kI8MapCache = 256;
-I8MapCacheEntry g_i8_maps[kI8MapCache];
-int g_i8_maps_used = 0, g_i8_maps_next = 0;
-std::mutex g_i8_maps_mu;
-
-int encode_i8_maps(const uint32_t* qw, int64_t qw_rows, const uint16_t* scales, int G, int N, I8Maps* maps) {
+// Maps over qw [qw_rows][N] uint32 with boxes of 256 columns x 2^i rows.
+int make_int_maps(const uint32_t* qw, int64_t qw_rows, int N, IntMaps* maps) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return QGEMM_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)qw_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
     const cuuint32_t estr[2] = {1, 1};
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)qw_rows};
-        const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
-        for (int i = 0; i < kI8BoxMaps; ++i) {
-            const cuuint32_t box[2] = {(cuuint32_t)kI8TileCols, (cuuint32_t)(1u << i)};
-            const CUresult r = fn(&maps->w[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qw), dims,
-                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-            if (r != CUDA_SUCCESS) return QGEMM_ERR_CUDA;
-        }
+    for (int i = 0; i < kIntBoxMaps; ++i) {
+        const cuuint32_t box[2] = {(cuuint32_t)kGemvTileCols, (cuuint32_t)(1u << i)};
+        const CUresult r = fn(&maps->box[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(qw), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return QGEMM_ERR_CUDA;
     }
-    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)G};
-    const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kI8TileCols, 2u};  // the two groups of a unit
-    const CUresult r = fn(&maps->s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(scales), dims, strides,
-                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? QGEMM_OK : QGEMM_ERR_CUDA;
-}
-
-int get_i8_maps(int dev, const uint32_t* qw, int64_t qw_rows, const uint16_t* scales, int G, int N, I8Maps* out) {
-    {
-        std::lock_guard<std::mutex> lk(g_i8_maps_mu);
-        for (int i = 0; i < g_i8_maps_used; ++i) {
-            const I8MapCacheEntry& e = g_i8_maps[i];
-            if (e.dev == dev && e.qw == qw && e.sc == scales && e.rows == qw_rows && e.n == N && e.g == G) {
-                *out = e.maps;
-                return QGEMM_OK;
-            }
-        }
-    }
-    I8Maps m;
-    const int st = encode_i8_maps(qw, qw_rows, scales, G, N, &m);
-    if (st != QGEMM_OK) return st;
-    std::lock_guard<std::mutex> lk(g_i8_maps_mu);
-    I8MapCacheEntry& e = g_i8_maps[g_i8_maps_next];
-    e.dev = dev;
-    e.qw = qw;
-    e.sc = scales;
-    e.rows = qw_rows;
-    e.n = N;
-    e.g = G;
-    e.maps = m;
-    g_i8_maps_next = (g_i8_maps_next + 1) % kI8MapCache;
-    if (g_i8_maps_used < kI8MapCache) ++g_i8_maps_used;
-    *out = m;
     return QGEMM_OK;
 }
 
-// Slice counts tried above the smallest that fits.
-constexpr int kI8SliceSearch = 6;
-
-struct I8Plan {
-    int S = 1, cps = 1, grid = 1, maxt = 1, bcap = 1, ring = 0, mp = 1;
-    size_t smem = 0;
+// Workspace: [tickets][partial slots][activation records].
+struct IntWs {
+    size_t tickets, slots, rec, total;
 };
 
-// Blocks a slice can hold at most: a slice's rows exceed W/S by less than one
-// block (8 rows), and every block has at least 2 rows.
-int64_t i8_slice_blocks(int nb, int64_t W, int S) {
-    if (S == 1) return nb;
-    return std::min<int64_t>(nb, ((W + S - 1) / S + 8) / 2 + 1);
-}
-
-// Slices S: the fewest whose activation tiles fit kI8MaxBlocks, then among a
-// few more the one that keeps most SMs busy (S * floor(sms / S) CTAs) with the
-// fewest contributions per tile.  CTAs per slice are also capped so that every
-// CTA's share of the slice is at least one unit (the reduction relies on it).
-int plan_i8(int M, int K, int N, int64_t W, int sms, I8Plan* pl) {
+IntWs int_ws_layout(int M, int K, int N, int sms) {
+    const int mp = int_mp(M);
     const int nb = K / kBlockRows;
-    const int64_t T = (N + kI8TileCols - 1) / kI8TileCols;
-    int smin = 1;
-    while (smin <= kI8MaxSlices && i8_slice_blocks(nb, W, smin) > kI8MaxBlocks) ++smin;
-    if (smin > kI8MaxSlices) return QGEMM_ERR_UNSUPPORTED;
-    double best = 1e30;
-    int bS = 0, bC = 0;
-    const int64_t smax = std::min<int64_t>({(int64_t)smin + kI8SliceSearch, (int64_t)kI8MaxSlices, (int64_t)nb,
-                                            std::max<int64_t>(1, W / 8)});
-    for (int64_t S = smin; S <= std::max<int64_t>(smin, smax); ++S) {
-        if (i8_slice_blocks(nb, W, (int)S) > kI8MaxBlocks) continue;
-        const int64_t cap = sms / S;
-        if (cap < 1) break;
-        const int64_t rows = W / S - 8;
-        const int64_t work = rows > 0 ? T * rows / (64 + kI8UnitCost) : 1;  // a unit: 2 groups of <= 32 rows
-        const int64_t cps = std::max<int64_t>(1, std::min<int64_t>(cap, work));
-        const double eff = (double)(S * cps) / sms;
-        const double score = (1.0 / eff) * (1.0 + 0.004 * S);
-        if (score < best) {
-            best = score;
-            bS = (int)S;
-            bC = (int)cps;
-        }
-    }
-    if (bS == 0) return QGEMM_ERR_UNSUPPORTED;
-    pl->S = bS;
-    pl->cps = bC;
-    pl->grid = bS * bC;
-    pl->maxt = (int)(T / bC) + 3;
-    pl->bcap = (int)i8_slice_blocks(nb, W, bS);
-    pl->mp = i8_mp(M);
-    pl->maxt = (int)(T / bC) + 3;
-    const I8Smem L0 = i8_smem_layout(nb, bS, pl->bcap, 0, pl->mp, pl->maxt);
-    const int64_t budget = 227 * 1024;
-    const int64_t ring = (budget - L0.total) / kI8RowBytes;
-    if (ring < 2 * (1 + 8 * 8)) return QGEMM_ERR_UNSUPPORTED;  // two units of 8 blocks of 8 rows
-    pl->ring = (int)std::min<int64_t>(ring, 1024);
-    pl->smem = (size_t)i8_smem_layout(nb, bS, pl->bcap, pl->ring, pl->mp, pl->maxt).total;
-    return QGEMM_OK;
-}
-
-// Workspace: [tickets per tile][partial sums per (CTA, local tile)].
-struct I8Ws {
-    size_t tickets, partial, total;
-};
-
-I8Ws i8_ws_layout(int M, int N, const I8Plan& pl) {
-    const size_t T = (N + kI8TileCols - 1) / kI8TileCols;
-    I8Ws w;
+    IntWs w;
     w.tickets = 0;
-    w.partial = align_up(T * 4, 256);
-    w.total = w.partial + (size_t)pl.grid * pl.maxt * pl.mp * kI8TileCols * 4;
-    (void)M;
+    w.slots = align_up((size_t)gemv_tiles(N) * 4, 256);
+    w.rec = w.slots + align_up((size_t)gemv_max_grid(K, N, sms) * 2 * mp * kGemvTileCols * 4, 256);
+    w.total = w.rec + align_up((size_t)(nb + 8) * int_rec_bytes(mp), 256);
     return w;
 }
 
-// Workspace bytes that every schedule of this shape fits (qgemm_workspace_bytes
-// does not see the schedule): grid * maxt <= S * T + 3 * sms with S at most
-// the largest slice count any word-row total can choose.
-size_t i8_ws_bound(int M, int K, int N, int sms) {
+// Two CTAs per SM for M <= 2 (one for M <= 4, whose activations need more
+// registers); grid capped as for the tensor-core GEMV so that every CTA's
+// range holds at least one unit.
+int plan_int(int M, int K, int N, int64_t qw_rows, int sms, GemvPlan* plan, int* cps_out) {
     const int nb = K / kBlockRows;
-    const int64_t T = (N + kI8TileCols - 1) / kI8TileCols;
-    int smin = 1;
-    while (smin < kI8MaxSlices && i8_slice_blocks(nb, 8 * (int64_t)nb, smin) > kI8MaxBlocks) ++smin;
-    const int64_t smax = std::min<int64_t>({(int64_t)smin + kI8SliceSearch, (int64_t)kI8MaxSlices, (int64_t)nb});
-    const int64_t slots = smax * T + 3 * (int64_t)sms;
-    return align_up((size_t)T * 4, 256) + (size_t)slots * i8_mp(M) * kI8TileCols * 4;
+    const int mp = int_mp(M);
+    const int cps = int_ctas_per_sm(mp);
+    // units of two 128-row groups: cost = word rows + 1, at most 8 * 8 + 1
+    const int64_t nu = (nb + kIntUnitBlocks - 1) / kIntUnitBlocks;
+    const int64_t U = (int64_t)gemv_tiles(N) * nu;
+    const int64_t C = (int64_t)gemv_tiles(N) * (qw_rows + nu);
+    const int64_t gcap = std::max<int64_t>(1, C / (8 * kIntUnitBlocks + 2));
+    const int64_t G = std::min<int64_t>(std::min<int64_t>(U, gcap), (int64_t)cps * sms);
+    const size_t fixed = int_fixed_smem(nb, mp);
+    const size_t budget = (size_t)(cps == 2 ? 113 : 227) * 1024;
+    if (fixed + (size_t)kGemvMinRing * kIntRowBytes > budget) return QGEMM_ERR_UNSUPPORTED;
+    const int ring = (int)std::min<size_t>(kGemvMaxRing, (budget - fixed) / kIntRowBytes);
+    plan->grid = (int)G;
+    plan->ring = ring;
+    plan->span_cap = 0;
+    plan->smem = fixed + (size_t)ring * kIntRowBytes;
+    if (cps_out) *cps_out = cps;
+    return QGEMM_OK;
 }
 
 template <int MP>
-cudaError_t launch_i8(const I8Plan& plan, const I8Params& p, const I8Maps& maps, cudaStream_t stream,
-                      bool* attr_done) {
+cudaError_t launch_int(const GemvPlan& plan, const IntParams& p, const IntMaps& maps, cudaStream_t stream,
+                       bool* attr_done) {
     if (!*attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_i8_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemv_int_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              227 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemv_int_kernel<MP>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         *attr_done = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.grid);
-    cfg.blockDim = dim3(kI8Threads);
+    cfg.blockDim = dim3(kIntThreads);
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -407,46 +312,72 @@ cudaError_t launch_i8(const I8Plan& plan, const I8Params& p, const I8Maps& maps,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_i8_kernel<MP>, p, maps);
+    return cudaLaunchKernelEx(&cfg, gemv_int_kernel<MP>, p, maps);
 }
 
-int run_gemv_i8(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
-                const uint16_t* scales, const uint8_t* bits, const int32_t* offs, int M, int K, int N, uint16_t* y,
-                void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev) {
-    int devid = 0;
-    if (cudaGetDevice(&devid) != cudaSuccess) return QGEMM_ERR_CUDA;
-    I8Plan plan;
-    int st = plan_i8(M, K, N, qw_rows, dev->sms, &plan);
+int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
+                 const uint16_t* scales, const uint8_t* bits, const int32_t* offs, int M, int K, int N,
+                 uint16_t* y, void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev) {
+    GemvPlan plan;
+    int st = plan_int(M, K, N, qw_rows, dev->sms, &plan, nullptr);
     if (st != QGEMM_OK) return st;
-    const I8Ws L = i8_ws_layout(M, N, plan);
-    if (ws == nullptr || ws_bytes < L.total) return QGEMM_ERR_WORKSPACE;
-    I8Maps maps;
-    const int G = (K + kGroupRows - 1) / kGroupRows;
-    if ((st = get_i8_maps(devid, qw, qw_rows, scales, G, N, &maps)) != QGEMM_OK) return st;
+    const IntWs L = int_ws_layout(M, K, N, dev->sms);
+    if (ws_bytes < L.total || ws == nullptr) return QGEMM_ERR_WORKSPACE;
+    IntMaps maps;
+    if ((st = make_int_maps(qw, qw_rows, N, &maps)) != QGEMM_OK) return st;
     uint8_t* w8 = static_cast<uint8_t*>(ws);
-    I8Params p;
-    p.x = x;
-    p.perm = perm;
+    const int nb = K / kBlockRows;
+    const int mp = int_mp(M);
+
+    IntPrepParams xp;
+    xp.x = x;
+    xp.perm = perm;
+    xp.bits = bits;
+    xp.rec = w8 + L.rec;
+    xp.M = M;
+    xp.K = K;
+    xp.nb = nb;
+    xp.mp = mp;
+    xp.x_bf16 = (x_dtype == QGEMM_BF16);
+    {
+        // programmatic dependent of the previous grid (it waits for it on the
+        // device), so its launch overlaps that grid's tail
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((nb + 7) / 8);
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, xprep_int_kernel, xp) != cudaSuccess) {
+            cudaGetLastError();
+            return QGEMM_ERR_CUDA;
+        }
+    }
+
+    IntParams p;
+    p.rec = xp.rec;
+    p.qw = qw;
+    p.qw_rows = qw_rows;
+    p.scales = reinterpret_cast<const __half*>(scales);
     p.bits = bits;
     p.offs = offs;
-    p.qw_rows = qw_rows;
     p.y = reinterpret_cast<__half*>(y);
     p.tickets = reinterpret_cast<int*>(w8 + L.tickets);
-    p.partial = reinterpret_cast<float*>(w8 + L.partial);
+    p.slots = reinterpret_cast<float*>(w8 + L.slots);
     p.M = M;
     p.K = K;
     p.N = N;
-    p.nb = K / kBlockRows;
-    p.tiles = (N + kI8TileCols - 1) / kI8TileCols;
-    p.S = plan.S;
-    p.cps = plan.cps;
-    p.maxt = plan.maxt;
+    p.nb = nb;
+    p.ng = gemv_groups(K);
+    p.tiles = gemv_tiles(N);
     p.ring_rows = plan.ring;
-    p.bcap = plan.bcap;
-    p.x_bf16 = (x_dtype == QGEMM_BF16);
-    const cudaError_t e = (plan.mp == 1)   ? launch_i8<1>(plan, p, maps, stream, &dev->i8_attr[0])
-                          : (plan.mp == 2) ? launch_i8<2>(plan, p, maps, stream, &dev->i8_attr[1])
-                                           : launch_i8<4>(plan, p, maps, stream, &dev->i8_attr[2]);
+    // programmatic dependent of xprep_int, as for the tensor-core GEMV
+    const cudaError_t e = (mp == 1)   ? launch_int<1>(plan, p, maps, stream, &dev->int_attr[0])
+                          : (mp == 2) ? launch_int<2>(plan, p, maps, stream, &dev->int_attr[1])
+                                      : launch_int<4>(plan, p, maps, stream, &dev->int_attr[2]);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return QGEMM_ERR_CUDA;
@@ -704,7 +635,7 @@ size_t qgemm_workspace_bytes(int M, int K, int N) {
     DeviceInfo* dev = nullptr;
     const int sms = (current_device_info(&dev) == QGEMM_OK) ? dev->sms : 148;
     const int path = qgemm_path_for(M, K, N);
-    if (path == kPathGemvInt) return i8_ws_bound(M, K, N, sms);
+    if (path == kPathGemvInt) return int_ws_layout(M, K, N, sms).total;
     if (path == kPathGemvTc) return gemv_ws_layout(M, K, N, sms).total;
     return gemm_ws_layout(M, K, N, sms).total;
 }
@@ -721,11 +652,12 @@ int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out) {
     out[0] = qgemm_path_for(M, K, N);
     out[5] = sms;
     if (out[0] == kPathGemvInt) {
-        I8Plan plan;
-        if ((st = plan_i8(M, K, N, qw_rows, sms, &plan)) != QGEMM_OK) return st;
+        GemvPlan plan;
+        int cps = 1;
+        if ((st = plan_int(M, K, N, qw_rows, sms, &plan, &cps)) != QGEMM_OK) return st;
         out[1] = plan.grid;
         out[2] = plan.ring;
-        out[3] = 1;
+        out[3] = cps;
         out[4] = (int64_t)plan.smem;
         return QGEMM_OK;
     }
@@ -805,8 +737,8 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm, const uint32_t* d
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int path = qgemm_path_for(M, K, N);
     if (path == kPathGemvInt)
-        return run_gemv_i8(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y, d_ws,
-                           ws_bytes, s, dev);
+        return run_gemv_int(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y,
+                            d_ws, ws_bytes, s, dev);
     if (path == kPathGemvTc)
         return run_gemv(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y,
                         d_ws, ws_bytes, s, dev);
@@ -829,20 +761,18 @@ int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm, co
         return QGEMM_ERR_ALIGN;
     DeviceInfo* dev = nullptr;
     if ((st = current_device_info(&dev)) != QGEMM_OK) return st;
-    I8Plan plan;
-    if ((st = plan_i8(M, K, N, qw_rows, dev->sms, &plan)) != QGEMM_OK) return st;
-    const I8Ws L = i8_ws_layout(M, N, plan);
+    const IntWs L = int_ws_layout(M, K, N, dev->sms);
     if (L.total > QGEMM_NOALLOC_SCRATCH_BYTES) return QGEMM_ERR_WORKSPACE;
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != QGEMM_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the tickets (the layout's first bytes, up to the partial sums) must start at zero
-    if (cudaMemsetAsync(scratch, 0, L.partial, s) != cudaSuccess) {
+    // the tickets (the layout's first bytes, up to the partial-sum slots) must start at zero
+    if (cudaMemsetAsync(scratch, 0, L.slots, s) != cudaSuccess) {
         cudaGetLastError();
         return QGEMM_ERR_CUDA;
     }
-    return run_gemv_i8(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y, scratch,
-                       QGEMM_NOALLOC_SCRATCH_BYTES, s, dev);
+    return run_gemv_int(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y, scratch,
+                        QGEMM_NOALLOC_SCRATCH_BYTES, s, dev);
 }
 
 }  // extern "C"

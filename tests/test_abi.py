@@ -197,3 +197,15 @@ def test_pack_and_dequant_reject_mismatched_shapes():
     with pytest.raises(ValueError):
         q.qgemm_dequant(a["qw"], torch.zeros(3, 64, dtype=torch.float16), a["bits"], a["offs"],
                         torch.zeros(256, 64, dtype=torch.float16))
+
+
+def test_noalloc_scratch_size_agrees_and_serves_every_decode_shape():
+    """The binding's copy of QGEMM_NOALLOC_SCRATCH_BYTES is the header's, and
+    the largest decode shape the ABI accepts (M = 4, K = 65536, N = 2^24)
+    needs no more scratch than the built-in buffer holds."""
+    text = open(HEADER).read()
+    m = re.search(r"#define QGEMM_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert m, "header constant not found"
+    assert int(m.group(1)) << int(m.group(2)) == q.NOALLOC_SCRATCH_BYTES
+    for M in (1, 2, 3, 4):
+        assert q.qgemm_workspace_bytes(M, 65536, 1 << 24) <= q.NOALLOC_SCRATCH_BYTES

@@ -1,8 +1,8 @@
-"""Host-side checks of the tensor-core GEMV launch plan (5 <= M <= 16), without
-a GPU.
+"""Host-side checks of the decode GEMV launch plan, without a GPU.
 
-The kernel (csrc/gemv.cuh) splits the (256-column tile, 128-row group) units
-into contiguous, equal-cost ranges, one per CTA.  This file replays that
+Both decode kernels (csrc/gemv_int.cuh for M <= 4, csrc/gemv.cuh for M <= 16)
+split the (256-column tile, 128-row group) units into contiguous, equal-cost
+ranges, one per CTA.  This file replays that
 split in Python for the workload shapes and checks what keeps the kernel in
 bounds: every unit is owned by exactly one CTA, the CTA that owns a unit is the
 one the reducer expects (cta_of), a unit fits the shared-memory ring, and partial-sum slots stay
@@ -59,7 +59,7 @@ def shapes():
     return out
 
 
-@pytest.mark.parametrize("M", [5, 8, 9, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 9, 16])
 @pytest.mark.parametrize("case", shapes(), ids=lambda c: f"{c[0]}-{c[1]}x{c[2]}")
 def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     name, K, N, bits = case
@@ -70,12 +70,15 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     plan = q.qgemm_plan_info(M, K, N, rows)
     if plan["path"] == 2:
         pytest.skip("this shape's M runs the split-k GEMM")
-    assert plan["path"] == 1
-    integer = False
+    integer = plan["path"] == 0
     G = plan["grid"]
     cps = plan["ctas_per_sm"]
-    mp = 8 if M <= 8 else 16
-    assert cps == 1                          # each CTA holds all of TMEM
+    if integer:
+        mp = 1 if M == 1 else 2 if M == 2 else 4 if M <= 4 else 8 if M <= 8 else 16
+        assert cps == (2 if mp <= 2 else 1)
+    else:
+        mp = 8 if M <= 8 else 16
+        assert cps == 1                          # each CTA holds all of TMEM
     assert 1 <= G <= cps * plan["sms"]
     # resident CTAs fit the SM's 228 KB (1 KB reserved per CTA)
     assert cps * (plan["smem"] + 1024) <= 228 * 1024
@@ -86,7 +89,7 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     assert all(a <= b for a, b in zip(starts, starts[1:]))
     ws = q.qgemm_workspace_bytes(M, K, N)
     slot_bytes = mp * TILE * 4
-    rec = (72 * mp + 15) // 16 * 16 if integer else 64 * mp
+    rec = (140 * mp + 4 + 15) // 16 * 16 if integer else 64 * mp   # integer: two int16 parts, three int32 arrays, a flag
     act_bytes = nb * rec + (0 if integer else ((nb + 3) // 4) * mp * 4 + 64)
     assert ws >= ((tiles * 4 + 255) // 256 * 256) + G * 2 * slot_bytes + act_bytes
     rng = np.random.default_rng(K + N + M)
@@ -109,7 +112,7 @@ def test_gemv_plan_keeps_kernel_in_bounds(case, M):
     assert need <= plan["ring"]
 
 
-def ring_progress(rows_seq, R, slots):
+def ring_progress(rows_seq, R, slots=16):
     """Replay the producer's admission rule with the consumers releasing units
     in order only when asked: every unit must be admitted at the latest once all
     earlier units are released (no wait that can never end)."""
@@ -133,17 +136,17 @@ def ring_progress(rows_seq, R, slots):
 
 @pytest.mark.parametrize("M", [1, 2, 4])
 @pytest.mark.parametrize("case", shapes(), ids=lambda c: f"{c[0]}-{c[1]}x{c[2]}")
-def test_integer_mma_gemv_ring_always_admits(case, M):
-    """The integer tensor-core GEMV's ring: a unit is its scale row plus the
-    word rows of two group parts (at most 8 blocks of 8 rows); 32 units in
-    flight."""
+def test_integer_gemv_ring_always_admits(case, M):
     name, K, N, bits = case
     offs = W.offsets(bits)
     nb = K // 32
     plan = q.qgemm_plan_info(M, K, N, int(offs[-1]))
     assert plan["path"] == 0
+    mp = 1 if M == 1 else 2 if M == 2 else 4 if M <= 4 else 8 if M <= 8 else 16
+    rec = (140 * mp + 4 + 15) // 16 * 16   # two int16 parts, three int32 arrays, a flag
     nu = (nb + 7) // 8
-    rows = [1 + int(offs[min(8 * g + 8, nb)] - offs[8 * g]) for g in range(nu)]
+    rows = [1 + int(offs[min(8 * g + 8, nb)] - offs[8 * g]) + -(-min(8, nb - 8 * g) * rec // 1024)
+            for g in range(nu)]
     seq = rows * 3                      # a CTA range can run over several tiles
     for start in range(0, nu, max(1, nu // 8)):
-        ring_progress(seq[start:start + 2 * nu], plan["ring"], 32)
+        ring_progress(seq[start:start + 2 * nu], plan["ring"])

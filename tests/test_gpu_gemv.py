@@ -167,7 +167,7 @@ def test_gemv_deterministic_and_workspace_reset(q):
         ys.append(y)
     torch.cuda.synchronize()
     assert all(torch.equal(ys[0], t) for t in ys[1:])
-    tickets = ws[: (N + 255) // 256 * 4].view(torch.int32)   # one ticket per 256-column tile
+    tickets = ws[: (N + 255) // 256 * 4].view(torch.int32)
     assert int(tickets.abs().sum()) == 0
 
 
