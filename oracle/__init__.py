@@ -16,6 +16,8 @@ Functions (all numpy in, numpy out):
 * ``dequant_f16(qw, scales, bits, K)``   RNE fp16 weights (uint16 bits)
 * ``qgemm_f64(x, perm, qw, scales, bits, cols=None, threads=0)``
       y = x[:, perm] . dequant(qw), double [M, N] (or [M, len(cols)])
+* ``quantize(w, bits, threads=0)``  fp16 W [K, N] -> codes, fp16 scales, the
+      chosen candidate, the 96 candidate errors and the per-column errors
 
 Parity pins for every function are in ``tests/test_oracle.py``.
 """
@@ -47,7 +49,7 @@ def build(force: bool = False) -> str:
             if f.read().strip() == h:
                 return _LIB
     tmp = _LIB + f".tmp{os.getpid()}"
-    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC,
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-o", tmp, _SRC,
                            "-lm", "-lpthread"])
     os.replace(tmp, _LIB)
     with open(_STAMP, "w") as f:
@@ -70,6 +72,8 @@ def _bind(lib):
     lib.oracle_qgemm_f64.restype = ctypes.c_int
     lib.oracle_qgemm_f64.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                      P, ctypes.c_int64, P, ctypes.c_int]
+    lib.oracle_quantize.restype = ctypes.c_int
+    lib.oracle_quantize.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P, P, P, P, ctypes.c_int]
     lib.oracle_half_to_double_n.restype = None
     lib.oracle_half_to_double_n.argtypes = [P, P, ctypes.c_int64]
     lib.oracle_double_to_half_n.restype = None
@@ -83,7 +87,7 @@ def compile_variant(src_text: str, out_path: str) -> str:
     c_path = out_path + ".c"
     with open(c_path, "w") as f:
         f.write(src_text)
-    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", out_path, c_path,
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-o", out_path, c_path,
                            "-lm", "-lpthread"])
     return out_path
 
@@ -196,6 +200,32 @@ class Oracle:
                                                cp, nc, _ptr(y), threads), "qgemm_f64")
         return y, used
 
+    def quantize(self, w, bits, threads: int = 0) -> "Quantized":
+        """fp16 W [K, N] (np.float16 or uint16 bit patterns) -> codes, scales."""
+        wa = np.asarray(w)
+        wb = _c(wa.view(np.uint16) if wa.dtype == np.float16 else wa, np.uint16)
+        b = _c(bits, np.uint8)
+        K, N = wb.shape
+        G = (K + 127) // 128
+        codes = np.empty((K, N), dtype=np.uint8)
+        scales = np.empty((G, N), dtype=np.uint16)
+        colerr = np.empty((96, N), dtype=np.float64)
+        err = np.empty(96, dtype=np.float64)
+        best = _check(self.lib.oracle_quantize(_ptr(wb), _ptr(b), K, N, _ptr(codes), _ptr(scales),
+                                               _ptr(colerr), _ptr(err), threads), "quantize")
+        return Quantized(codes, scales, best, err, colerr)
+
+
+class Quantized:
+    """Result of the oracle's quantiser."""
+
+    def __init__(self, codes, scales, best, err, colerr):
+        self.codes = codes        # uint8 [K, N]
+        self.scales = scales      # fp16 bit patterns, uint16 [G, N]
+        self.best = best          # chosen candidate index (p = (32 + best) / 96)
+        self.err = err            # double [96]: E(p_i)
+        self.colerr = colerr      # double [96, N]: per-column errors
+
 
 def get() -> Oracle:
     """The oracle built from oracle.c as it stands."""
@@ -234,6 +264,10 @@ def dequant_f64(qw, scales, bits, K):
 
 def dequant_f16(qw, scales, bits, K):
     return get().dequant_f16(qw, scales, bits, K)
+
+
+def quantize(w, bits, threads=0):
+    return get().quantize(w, bits, threads)
 
 
 def qgemm_f64(x, perm, qw, scales, bits, cols=None, threads=0):

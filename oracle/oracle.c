@@ -268,3 +268,168 @@ void oracle_half_to_double_n(const uint16_t *h, double *v, int64_t n) {
 void oracle_double_to_half_n(const double *v, uint16_t *h, int64_t n) {
     for (int64_t i = 0; i < n; ++i) h[i] = oracle_double_to_half(v[i]);
 }
+
+/* ---------------------------------------------------------------------------
+ * Quantiser: fp16 weights W [K][N] (act-order rows) and the block widths ->
+ * codes [K][N] and fp16 scales [ceil(K/128)][N], the step before pack.
+ *
+ * The pages (nightvoyager.top exllamav2 report, "关键设计决策", adaptive scale
+ * paragraph) name two parts: a 4-bit second-level quantisation of the group
+ * scale, qscale = round(sqrt(base_scale / qscale_max) * (scale_maxq + 1)), and
+ * a scan of 96 candidate p factors per layer that keeps the one with the
+ * lowest quantisation error.  Everything else is this library's reading:
+ *
+ *   base[g]  = max over the blocks j of group g of max_k |W[k][n]| / 2^(b_j-1)
+ *              (the smallest scale at which no weight of the group exceeds
+ *              its block's largest code magnitude);
+ *   qmax     = max_g base[g] (per column);
+ *   qs[g]    = clamp(rint(sqrt(base[g] / qmax) * 16), 1, 16), the 4-bit
+ *              second-level scale (scale_maxq = 15);
+ *   p_i      = (32 + i) / 96, i = 0..95 (p_64 = 1);
+ *   s_i[g]   = fp16(p_i * (qmax * (qs[g]^2 / 256)));
+ *   q        = clamp(rint(W * (1 / s)) + 2^(b-1), 0, 2^b - 1), and q = 2^(b-1)
+ *              where s is 0 (an all-zero column);
+ *   e        = (W - (q - 2^(b-1)) * s)^2;
+ *   E(p_i)   = sum over columns n (increasing) of the sum over rows k
+ *              (increasing) of e; the layer keeps the smallest E (the lowest
+ *              i on ties) and those codes and scales.
+ * Arithmetic: single precision, each operation rounded to nearest even (the
+ * precision the GPU kernel decides codes in), the error terms and sums in
+ * double.  fp16 <-> float conversions go through the exact helpers above.
+ * ------------------------------------------------------------------------- */
+#define ORC_QCANDS 96
+
+static float cand_factor(int i) { return (float)(32 + i) / 96.0f; }
+
+static float half_to_float(uint16_t h) { return (float)oracle_half_to_double(h); }
+
+/* 4-bit second-level scales qs[g] (as floats 1..16) and qmax of column n. */
+static float column_qscales(const uint16_t *w, const uint8_t *bits, int K, int64_t N, int64_t n, float *qs) {
+    int G = (K + ORC_GROUP - 1) / ORC_GROUP;
+    float qmax = 0.0f;
+    for (int g = 0; g < G; ++g) {
+        float base = 0.0f;
+        for (int k = g * ORC_GROUP; k < K && k < (g + 1) * ORC_GROUP; ++k) {
+            float a = fabsf(half_to_float(w[(int64_t)k * N + n]));
+            float r = a / (float)(1 << (bits[k / ORC_BLOCK] - 1));  /* exact: a power of two */
+            if (r > base) base = r;
+        }
+        qs[g] = base;  /* base for now */
+        if (base > qmax) qmax = base;
+    }
+    for (int g = 0; g < G; ++g) {
+        if (qmax == 0.0f) {
+            qs[g] = 16.0f;
+            continue;
+        }
+        float t = rintf(sqrtf(qs[g] / qmax) * 16.0f);
+        qs[g] = t < 1.0f ? 1.0f : (t > 16.0f ? 16.0f : t);
+    }
+    return qmax;
+}
+
+static uint16_t cand_scale(float p, float qmax, float qs) {
+    float u = qmax * ((qs * qs) / 256.0f);  /* qs^2 exact, /256 exact */
+    float v = p * u;
+    return oracle_double_to_half((double)v);
+}
+
+/* Codes of column n under the given group scales; returns the squared error
+ * summed over k in increasing order. */
+static double column_codes(const uint16_t *w, const uint8_t *bits, int K, int64_t N, int64_t n,
+                           const uint16_t *sc, uint8_t *codes) {
+    double err = 0.0;
+    int g_cur = -1;
+    float s = 0.0f, inv = 0.0f;
+    for (int k = 0; k < K; ++k) {
+        int g = k / ORC_GROUP;
+        if (g != g_cur) {
+            g_cur = g;
+            s = half_to_float(sc[g]);
+            inv = (s == 0.0f) ? 0.0f : 1.0f / s;
+        }
+        int b = bits[k / ORC_BLOCK], z = 1 << (b - 1);
+        float x = half_to_float(w[(int64_t)k * N + n]);
+        int q = z;
+        if (s != 0.0f) {
+            float t = rintf(x * inv);
+            if (t != t) t = 0.0f;  /* not a number: the zero point */
+            float lo = (float)(-z), hi = (float)((1 << b) - 1 - z);
+            t = t < lo ? lo : (t > hi ? hi : t);
+            q = (int)t + z;
+        }
+        if (codes) codes[(int64_t)k * N + n] = (uint8_t)q;
+        double d = (double)x - (double)((float)(q - z) * s);
+        err += d * d;
+    }
+    return err;
+}
+
+typedef struct {
+    const uint16_t *w; const uint8_t *bits; int K; int64_t N, c0, c1; double *colerr;
+} quant_job;
+
+static void *quant_worker(void *arg) {
+    quant_job *J = (quant_job *)arg;
+    int G = (J->K + ORC_GROUP - 1) / ORC_GROUP;
+    float *qs = (float *)malloc(sizeof(float) * (size_t)G);
+    uint16_t *sc = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)G);
+    for (int64_t n = J->c0; n < J->c1; ++n) {
+        float qmax = column_qscales(J->w, J->bits, J->K, J->N, n, qs);
+        for (int i = 0; i < ORC_QCANDS; ++i) {
+            for (int g = 0; g < G; ++g) sc[g] = cand_scale(cand_factor(i), qmax, qs[g]);
+            J->colerr[(int64_t)i * J->N + n] = column_codes(J->w, J->bits, J->K, J->N, n, sc, NULL);
+        }
+    }
+    free(qs); free(sc);
+    return NULL;
+}
+
+/* w: fp16 bits [K][N]; codes: [K][N]; scales: fp16 bits [ceil(K/128)][N];
+ * colerr (optional): double [96][N], the error of every column under every
+ * candidate; err: double [96], E(p_i).  Returns the chosen candidate index
+ * (>= 0) or a negative error.  nthreads <= 0 uses every online core. */
+int oracle_quantize(const uint16_t *w, const uint8_t *bits, int K, int N, uint8_t *codes, uint16_t *scales,
+                    double *colerr, double *err, int nthreads) {
+    int64_t rows = oracle_word_rows(bits, K);
+    if (rows < 0) return (int)rows;
+    if (N <= 0) return ORC_ERR_SHAPE;
+    double *ce = colerr ? colerr : (double *)malloc(sizeof(double) * ORC_QCANDS * (size_t)N);
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > N) nthreads = N;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    quant_job *jobs = (quant_job *)malloc(sizeof(quant_job) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) {
+        quant_job J = {w, bits, K, N, (int64_t)N * t / nthreads, (int64_t)N * (t + 1) / nthreads, ce};
+        jobs[t] = J;
+        pthread_create(&th[t], NULL, quant_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+    free(th); free(jobs);
+    int best = 0;
+    double best_e = 0.0;
+    for (int i = 0; i < ORC_QCANDS; ++i) {
+        double e = 0.0;
+        for (int64_t n = 0; n < N; ++n) e += ce[(int64_t)i * N + n];
+        if (err) err[i] = e;
+        if (i == 0 || e < best_e) {
+            best = i;
+            best_e = e;
+        }
+    }
+    int G = (K + ORC_GROUP - 1) / ORC_GROUP;
+    float *qs = (float *)malloc(sizeof(float) * (size_t)G);
+    uint16_t *sc = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)G);
+    for (int64_t n = 0; n < N; ++n) {
+        float qmax = column_qscales(w, bits, K, N, n, qs);
+        for (int g = 0; g < G; ++g) {
+            sc[g] = cand_scale(cand_factor(best), qmax, qs[g]);
+            scales[(int64_t)g * N + n] = sc[g];
+        }
+        column_codes(w, bits, K, N, n, sc, codes);
+    }
+    free(qs); free(sc);
+    if (!colerr) free(ce);
+    return best;
+}

@@ -13,7 +13,12 @@ the oracle disagrees with the fact it checks.  The facts are:
 * a hand-written brute-force loop for y at K = 32, N = 1;
 * reduction to a dense numpy matmul for uniform widths and identity perm;
 * invariants: one-hot x, row permutation inside blocks, linearity,
-  per-row independence of x, column subsets.
+  per-row independence of x, column subsets;
+* the quantiser: weights built on its own grid come back exactly (codes,
+  scales, the p = 1 candidate, zero error); its error equals the squared
+  distance to the pinned dequantisation of its output; ties round to even;
+  an all-zero column gives zero-point codes and zero scales; codes stay
+  within each block's width and scales on the 16-level grid of the chosen p.
 
 ``tests/test_oracle.py`` runs them on the oracle and on copies of the oracle
 with planted mistakes, which must each fail at least one pin.
@@ -286,6 +291,102 @@ def pin_column_subset(o):
     cols = rng.choice(33, size=9, replace=False)
     yc, _ = o.qgemm_f64(x, perm, qw, s, bits, cols=cols)
     assert np.array_equal(yc, y[:, cols])
+
+
+# ------------------------------------------------------------- quantiser
+
+def _grid_problem(rng, bits, N):
+    """W exactly representable by the quantiser at p = 1: per column a power
+    of two S and per group qs in {4, 8, 12, 16} (one group at 16), scales
+    s = S qs^2 / 256, codes with at least one 0 per group (so the group's
+    largest |W| / 2^(b-1) is s)."""
+    bits = np.asarray(bits, dtype=np.uint8)
+    K = 32 * len(bits)
+    G = (K + 127) // 128
+    codes = np.empty((K, N), dtype=np.uint8)
+    for j, b in enumerate(bits):
+        codes[32 * j:32 * j + 32] = rng.integers(0, 1 << int(b), size=(32, N))
+    for g in range(G):
+        codes[128 * g + rng.integers(0, min(128, K - 128 * g)), :] = 0
+    qs = rng.choice([4, 8, 12, 16], size=(G, N))
+    qs[rng.integers(0, G, size=N), np.arange(N)] = 16
+    S = np.ldexp(1.0, rng.integers(-12, -4, size=N))
+    s = (S[None, :] * qs.astype(np.float64) ** 2 / 256.0).astype(np.float16)
+    assert np.array_equal(s.astype(np.float64), S[None, :] * qs.astype(np.float64) ** 2 / 256.0)
+    w = _w_from_codes(codes, bits, s).astype(np.float16)
+    assert np.array_equal(w.astype(np.float64), _w_from_codes(codes, bits, s))
+    return bits, codes, s, w
+
+
+def pin_quantize_grid_roundtrip(o):
+    rng = _rng(21)
+    bits = rng.choice(BITS, size=12).astype(np.uint8)
+    bits, codes, s, w = _grid_problem(rng, bits, 40)
+    r = o.quantize(w, bits)
+    assert r.best == 64                                     # p = 96/96 = 1
+    assert r.err[64] == 0.0 and (r.err[:64] > 0).all() and (r.err[65:] > 0).all()
+    assert np.array_equal(r.codes, codes)
+    assert np.array_equal(r.scales, s.view(np.uint16))
+
+
+def pin_quantize_error_is_distance_to_dequant(o):
+    rng = _rng(22)
+    bits = rng.choice(BITS, size=9).astype(np.uint8)
+    K, N = 32 * len(bits), 17
+    w = (rng.standard_normal((K, N)) * 0.03).astype(np.float16)
+    w[5, 3] = np.float16(0.9)                               # an outlier
+    r = o.quantize(w, bits)
+    wd = o.dequant_f64(o.pack(r.codes, bits), r.scales, bits, K)
+    d = w.astype(np.float64) - wd
+    col = np.array([np.cumsum(d[:, n] ** 2)[-1] for n in range(N)])
+    assert np.array_equal(col, r.colerr[r.best])            # same terms, same k order
+    assert r.err[r.best] == np.cumsum(col)[-1]
+    assert r.err[r.best] == r.err.min() and int(np.argmin(r.err)) == r.best
+    assert np.array_equal(r.err, np.array([np.cumsum(r.colerr[i])[-1] for i in range(96)]))
+
+
+def pin_quantize_ranges_and_scale_grid(o):
+    rng = _rng(23)
+    bits = rng.choice(BITS, size=16).astype(np.uint8)
+    K, N = 32 * len(bits), 24
+    w = (rng.standard_normal((K, N)) * np.exp(rng.standard_normal((1, N)))).astype(np.float16)
+    r = o.quantize(w, bits)
+    widths = np.repeat(bits.astype(np.int64), 32)[:, None]
+    assert (r.codes.astype(np.int64) < (1 << widths)).all()
+    p = np.float32(32 + r.best) / np.float32(96)
+    for n in range(N):
+        wf = np.abs(w[:, n].astype(np.float64)) / np.left_shift(1, widths[:, 0] - 1)
+        base = np.array([wf[128 * g:128 * g + 128].max() for g in range(r.scales.shape[0])])
+        grid = {o.double_to_half(np.array([float(np.float32(p) * np.float32(np.float32(base.max()) *
+                                                                         np.float32(q * q / 256.0)))]))[0]
+                for q in range(1, 17)}
+        assert set(r.scales[:, n].tolist()) <= grid
+
+
+def pin_quantize_ties_to_even_and_zero_column(o):
+    bits = np.array([8, 8, 8, 8], dtype=np.uint8)
+    K, N = 128, 3
+    q0 = np.tile(np.arange(128, dtype=np.int64)[:, None], (1, N))   # codes 0..127, z = 128
+    w = ((q0 - 128).astype(np.float64)).astype(np.float16)          # s = 1 at p = 1
+    w[10, 1] = np.float16(-117.5)                                   # between -118 and -117
+    w[11, 1] = np.float16(-116.5)                                   # between -117 and -116
+    w[:, 2] = 0
+    r = o.quantize(w, bits)
+    assert r.best == 64
+    assert r.scales[0, 0] == np.float16(1.0).view(np.uint16)
+    assert r.codes[10, 1] == 128 - 118 and r.codes[11, 1] == 128 - 116   # even neighbours
+    assert (r.codes[:, 2] == 128).all() and r.scales[0, 2] == 0 and r.colerr[:, 2].max() == 0.0
+
+
+def pin_quantize_ties_between_candidates_take_the_first(o):
+    """An all-zero layer has zero error under every candidate: the lowest
+    index wins, and the output is zero-point codes with zero scales."""
+    bits = np.array([2, 5, 3, 8, 6], dtype=np.uint8)
+    w = np.zeros((160, 9), dtype=np.float16)
+    r = o.quantize(w, bits)
+    assert r.best == 0 and (r.err == 0).all()
+    assert (r.codes == np.repeat(np.left_shift(1, bits - 1), 32)[:, None]).all()
+    assert (r.scales == 0).all()
 
 
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

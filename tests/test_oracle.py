@@ -55,6 +55,19 @@ MUTANTS = [
     ("code_check_dropped", "if (q >> b) return ORC_ERR_CODE;", "", 0),
     ("stream_bit_stride", "int64_t p = (int64_t)r * b + t;                 /* stream bit */",
      "int64_t p = (int64_t)r * (b + 1) + t;", 0),
+    # the quantiser
+    ("q_zero_point", "int b = bits[k / ORC_BLOCK], z = 1 << (b - 1);",
+     "int b = bits[k / ORC_BLOCK], z = (1 << (b - 1)) - 1;", 0),
+    ("q_base_width", "float r = a / (float)(1 << (bits[k / ORC_BLOCK] - 1));",
+     "float r = a / (float)(1 << bits[k / ORC_BLOCK]);", 0),
+    ("q_no_sqrt", "rintf(sqrtf(qs[g] / qmax) * 16.0f)", "rintf((qs[g] / qmax) * 16.0f)", 0),
+    ("q_qscale_levels", "rintf(sqrtf(qs[g] / qmax) * 16.0f)", "rintf(sqrtf(qs[g] / qmax) * 15.0f)", 0),
+    ("q_round_away", "float t = rintf(x * inv);", "float t = roundf(x * inv);", 0),
+    ("q_candidate_grid", "(float)(32 + i) / 96.0f", "(float)(33 + i) / 96.0f", 0),
+    ("q_argmin_last_tie", "if (i == 0 || e < best_e) {", "if (i == 0 || e <= best_e) {", 0),
+    ("q_clamp_high", "hi = (float)((1 << b) - 1 - z);", "hi = (float)((1 << b) - z);", 0),
+    ("q_group_of_row", "int g = k / ORC_GROUP;\n        if (g != g_cur) {",
+     "int g = k / ORC_BLOCK / 4 % 2;\n        if (g != g_cur) {", 0),
 ]
 
 
