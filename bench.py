@@ -9,18 +9,28 @@ weight, widths {2,3,4,5,6,8} per 32-row block, random act-order perm, fp16
 activations.  One step = one qgemm call.  Steps rotate over enough distinct
 weight copies (> 3x the 126 MB L2) that every step streams its weights from
 HBM; steps are captured in CUDA graphs and timed with CUDA events on the
-launching stream.
+launching stream: exactly K steps in one bracketed region give `value`.
 
 Extra objects on the same line:
-  roofline      the GEMV kernel against measured HBM bandwidth;
-  cpu_baseline  the CPU oracle timed on the host cores (rank 0, N = 1);
-  e2e           the same metric through the public call with host buffers
-                (x copied in from pinned memory, y copied back, every step);
+  roofline      the decode step against measured HBM bandwidth;
+  stats         the headline again as the interquartile mean (the 5/16 to
+                11/16 quantiles) of at least 200 graph replays lasting at
+                least 0.2 s in all;
+  configs       every benchmark configuration of the method, each with its
+                own roofline fraction, timed the same IQM way:
+                  single_4096x4096_u4      one 4096^2 layer, uniform 4-bit, M=1;
+                  decode_8192x28672_2p55   the headline layer at M = 2, 4, 8;
+                  llama70b_stack_2p5       80 layers x 7 Llama-3-70B linears,
+                                           M = 1, as tokens/s;
+                  sweep_8192x8192_3p75     M = 1 ... 512 on one 8192^2 layer,
+                                           the GEMV/GEMM crossover, with the
+                                           path each M dispatches to;
   prefill       TFLOP/s of the M = 2048 prefill GEMM (K = 8192, N = 28672,
                 4.0 bpw, bf16 activations) against the dense tensor peak;
-  decode_m_gbs, crossover_sweep, stack (with --full): other M of the headline
-                shape, the 8192 x 8192 M sweep that locates the GEMV/GEMM
-                crossover, and the 80-layer Llama-3-70B linear stack as tokens/s;
+  cpu_baseline  the CPU oracle timed on the host cores (rank 0, N = 1);
+  e2e           the headline metric through the public call with host
+                buffers (x copied in from pinned memory, y copied back, every
+                step), rotating the same weight copies, so HBM-bound too;
   clocks        SM clocks and throttle reasons sampled during the timed region.
 
 --impl reference times the CPU oracle (the only reference implementation this
@@ -54,7 +64,9 @@ SWEEP = "sweep_8192x8192_3p75"
 SWEEP_MS = (1, 2, 4, 8, 16, 32, 64, 128, 256, 512)
 STACK = "llama70b_stack_2p5"
 METRIC = "Q-GEMM weight GB/s at M=1 (% of HBM) and TFLOP/s at M=2048 (% of peak)"
+CFG1 = "single_4096x4096_u4"
 L2_BYTES = 126 * 1024 * 1024
+IQM_LO, IQM_HI = 5 / 16, 11 / 16
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -174,6 +186,17 @@ def max_over_ranks(v, ws):
     return float(t.item())
 
 
+
+
+def iqm(values, lo=IQM_LO, hi=IQM_HI):
+    """Mean of the values between the lo and hi quantiles (sorted, at least one)."""
+    v = sorted(values)
+    n = len(v)
+    a = min(n - 1, int(math.floor(n * lo)))
+    b = max(a + 1, int(math.ceil(n * hi)))
+    return float(sum(v[a:b]) / (b - a))
+
+
 # ------------------------------------------------------------ GPU problems
 
 class Layer:
@@ -199,9 +222,46 @@ class Layer:
         self.y = torch.empty(M, N, dtype=torch.float16, device=device)
         self.ws = q.workspace(M, K, N, device=device)
 
+    def copy_weights(self):
+        """Same problem, distinct weight and scale storage (and workspace)."""
+        import mixed_bitwidth_weight_b200 as q
+        L = Layer.__new__(Layer)
+        L.__dict__.update(self.__dict__)
+        L.qw = self.qw.clone()
+        L.scales = self.scales.clone()
+        L.ws = q.workspace(self.M, self.K, self.N)
+        return L
+
+    def weight_bytes(self):
+        return 4 * self.N * self.rows + 2 * ((self.K + 127) // 128) * self.N
+
+    def nbytes(self):
+        return call_bytes(self.K, self.N, self.M, self.rows, self.x.element_size())
+
     def call(self, q, x=None, y=None):
         q.qgemm(self.x if x is None else x, self.perm, self.qw, self.scales, self.bits, self.offs,
                 self.y if y is None else y, self.ws)
+
+
+def tune(q, L):
+    """The library's per-shape autotune (20 warm-up + 200 timed calls per
+    candidate variant) on this problem; returns the choice and the candidates'
+    IQM times."""
+    r = q.qgemm_autotune(L.x, L.perm, L.qw, L.scales, L.bits, L.offs, L.y, L.ws, warmup=20, iters=200)
+    torch.cuda.synchronize()
+    return {"path": r["path"], "path_name": q.PATH_NAMES[r["path"]], "knob": r["knob"],
+            "candidates_us": {f"{c['path']}/{c['knob']}": (round(c["us"], 3) if c["us"] is not None else None)
+                              for c in r["candidates"]}}
+
+
+def rotation(q, w, M):
+    """Copies of one problem whose weights together exceed 3x L2, so that a
+    call never finds its weights in L2 from an earlier call; the shape is
+    autotuned first on the first copy."""
+    base = Layer(w, M)
+    tuned = tune(q, base)
+    R = max(1, math.ceil((3 * L2_BYTES + 1) / base.weight_bytes()))
+    return [base] + [base.copy_weights() for _ in range(R - 1)], tuned
 
 
 def graph_of(fn, n):
@@ -220,7 +280,7 @@ def graph_of(fn, n):
 
 
 def run_steps(fn, steps, chunk):
-    """Replay graphs so that exactly `steps` calls of fn run."""
+    """Graphs whose replays run exactly `steps` calls of fn."""
     graphs = {}
 
     def get(n):
@@ -235,156 +295,201 @@ def run_steps(fn, steps, chunk):
     return [get(n) for n in plan]
 
 
-def time_graphs(graphs, ws):
+def spin_up(graph, secs=0.05):
+    """Untimed replays for about `secs` right before a timed region, so that
+    the clocks are up whatever the warm-up count."""
+    torch.cuda.synchronize()
+    t = time.time()
+    n = 0
+    while time.time() - t < secs or n < 2:
+        graph.replay()
+        n += 1
+        if n % 8 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+
+
+def time_region(graphs, ws):
+    """One timed region: barrier + synchronize on both sides, an event pair
+    around all replays, one event between replays (per-replay times)."""
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
     t0 = time.time()
-    e0.record(st)
-    for g in graphs:
+    ev[0].record(st)
+    for i, g in enumerate(graphs):
         g.replay()
-    e1.record(st)
+        ev[i + 1].record(st)
     torch.cuda.synchronize()
     t1 = time.time()
     barrier(ws)
-    return e0.elapsed_time(e1) / 1e3, t0, t1
+    per = [ev[i].elapsed_time(ev[i + 1]) / 1e3 for i in range(len(graphs))]
+    return ev[0].elapsed_time(ev[-1]) / 1e3, per, t0, t1
 
 
-def decode_copies(w, M, target_bytes):
-    one = call_bytes(w.K, w.N, M, W.target_word_rows(w.K // 32, w.target_bpw) if w.target_bpw
-                     else (w.K // 32) * w.uniform_bits)
-    return max(1, math.ceil(target_bytes / one))
+def iqm_time(fn, calls_per_replay, ws, min_replays=200, min_secs=0.2, warm_replays=20, max_replays=4000):
+    """Seconds per call of fn as the IQM of per-replay times: warm-up
+    replays, then batches of timed replays until there are at least
+    min_replays lasting at least min_secs in all."""
+    g = graph_of(fn, calls_per_replay)
+    for _ in range(warm_replays):
+        g.replay()
+    spin_up(g)
+    per, total, t0, t1 = [], 0.0, None, None
+    while len(per) < min_replays or (total < min_secs and len(per) < max_replays):
+        n = max(1, min_replays - len(per)) if len(per) < min_replays else min_replays
+        secs, p, a, b = time_region([g] * n, ws)
+        t0 = a if t0 is None else t0
+        t1 = b
+        per += p
+        total += secs
+    per_call = [p / calls_per_replay for p in per]
+    v = max_over_ranks(iqm(per_call), ws)
+    del g
+    return dict(secs=v, replays=len(per), calls_per_replay=calls_per_replay, timed_secs=round(total, 4),
+                t0=t0, t1=t1)
 
 
-def bench_decode(q, w, M, steps, warmup, ws, chunk=192):
-    """GB/s of one workload at M rows, rotating over copies > 3x L2."""
-    R = decode_copies(w, M, 3 * L2_BYTES + 1)
-    base = Layer(w, M)
-    layers = [base]
-    for r in range(1, R):                    # distinct copies of the weights (same values)
-        L = Layer.__new__(Layer)
-        L.__dict__.update(base.__dict__)
-        L.qw = base.qw.clone()
-        L.scales = base.scales.clone()
-        L.ws = q.workspace(M, base.K, base.N)
-        layers.append(L)
-    fn = lambda i: layers[i % R].call(q)  # noqa: E731
+def hbm_roofline(nbytes, secs, peak, src):
+    gbs = nbytes / secs / 1e9
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(gbs / peak, 4), "peak_source": src}
+
+
+def mixed_roofline(nbytes, flops, secs, pk):
+    """Roofline of a call that may be bound by either HBM or the tensor pipe:
+    the target time is the slower of bytes / HBM peak and flops / bf16 peak."""
+    t_hbm = nbytes / (pk["hbm"] * 1e9)
+    t_tc = flops / (pk["bf16"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    return {"bound": bound, "target_us": round(max(t_hbm, t_tc) * 1e6, 3),
+            "frac": round(max(t_hbm, t_tc) / secs, 4), "peak_source": pk["src"]}
+
+
+# ------------------------------------------------------------------- legs
+
+def bench_headline(q, w, steps, warmup, ws, chunk=192):
+    """Exactly `steps` decode calls (M = 1) in one bracketed region, rotating
+    over weight copies > 3x L2; the IQM statistic of the same call as well."""
+    rot, tuned = rotation(q, w, 1)
+    R = len(rot)
+    fn = lambda i: rot[i % R].call(q)  # noqa: E731
     wg = run_steps(fn, warmup, chunk)
     tg = run_steps(fn, steps, chunk)
     for g in wg:
         g.replay()
-    secs, t0, t1 = time_graphs(tg, ws)
-    secs = max_over_ranks(secs, ws)
-    nbytes = call_bytes(base.K, base.N, M, base.rows)
-    return dict(secs=secs, t0=t0, t1=t1, bytes=nbytes, rows=base.rows, copies=R,
-                gbs=nbytes * steps / secs / 1e9, us=secs / steps * 1e6, layer=base)
-
-
-def bench_prefill(q, w, M, steps, warmup, ws):
-    """TFLOP/s of the prefill GEMM, rotating over weight copies > 3x L2."""
-    base = Layer(w, M)
-    one = 4 * base.N * base.rows + 2 * ((base.K + 127) // 128) * base.N
-    R = max(1, math.ceil((3 * L2_BYTES + 1) / one))
-    layers = [base]
-    for r in range(1, R):
-        L = Layer.__new__(Layer)
-        L.__dict__.update(base.__dict__)
-        L.qw = base.qw.clone()
-        L.scales = base.scales.clone()
-        layers.append(L)
-    fn = lambda i: layers[i % R].call(q)  # noqa: E731
-    wg = run_steps(fn, warmup, 16)
-    tg = run_steps(fn, steps, 16)
-    for g in wg:
+    for g in {id(g): g for g in tg}.values():   # untimed first replay of each graph (upload)
         g.replay()
-    secs, t0, t1 = time_graphs(tg, ws)
+    spin_up(wg[-1])
+    secs, _, t0, t1 = time_region(tg, ws)
     secs = max_over_ranks(secs, ws)
-    flops = 2.0 * M * base.K * base.N
-    return dict(secs=secs, t0=t0, t1=t1, flops=flops, rows=base.rows, copies=R,
-                tflops=flops * steps / secs / 1e12, ms=secs / steps * 1e3, layer=base)
+    del wg, tg
+    nbytes = rot[0].nbytes()
+    st = iqm_time(fn, R * max(1, math.ceil(24 / R)), ws)
+    return dict(secs=secs, t0=t0, t1=t1, bytes=nbytes, rows=rot[0].rows, copies=R,
+                gbs=nbytes * steps / secs / 1e9, us=secs / steps * 1e6, rot=rot, stats=st, tuned=tuned)
 
 
-def bench_sweep(q, w, Ms, ws):
-    """Crossover sweep: one shape, several M; GB/s and TFLOP/s per M and the path used."""
+def bench_decode_leg(q, w, M, pk, ws):
+    rot, tuned = rotation(q, w, M)
+    R = len(rot)
+    st = iqm_time(lambda i: rot[i % R].call(q), R * max(1, math.ceil(24 / R)), ws)
+    nbytes = rot[0].nbytes()
+    out = {"M": M, "K": rot[0].K, "N": rot[0].N, "path": q.qgemm_path_for(M, rot[0].K, rot[0].N),
+           "us": round(st["secs"] * 1e6, 3), "value": round(nbytes / st["secs"] / 1e9, 1), "unit": "GB/s",
+           "bytes_per_call": nbytes, "weight_copies": R, "replays": st["replays"], "tuned": tuned,
+           "roofline": hbm_roofline(nbytes, st["secs"], pk["hbm"], pk["src"])}
+    del rot
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_prefill(q, w, M, pk, ws):
+    rot, tuned = rotation(q, w, M)
+    R = len(rot)
+    st = iqm_time(lambda i: rot[i % R].call(q), R, ws, min_replays=60, min_secs=0.3, warm_replays=5)
+    flops = 2.0 * M * rot[0].K * rot[0].N
+    tf = flops / st["secs"] / 1e12
+    out = dict(secs=st["secs"], t0=st["t0"], t1=st["t1"], flops=flops, rows=rot[0].rows, copies=R,
+               tflops=tf, ms=st["secs"] * 1e3, replays=st["replays"], nbytes=rot[0].nbytes(), tuned=tuned)
+    del rot
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_sweep(q, w, Ms, pk, ws):
+    """Crossover sweep: one shape, several M; GB/s, TFLOP/s, the roofline
+    fraction (the slower of the HBM and tensor bounds) and the path per M."""
     out = {}
     for M in Ms:
-        base = Layer(w, M)
-        one = call_bytes(base.K, base.N, M, base.rows)
-        R = max(1, math.ceil((3 * L2_BYTES + 1) / (4 * base.N * base.rows)))
-        layers = [base]
-        for r in range(1, R):
-            L = Layer.__new__(Layer)
-            L.__dict__.update(base.__dict__)
-            L.qw = base.qw.clone()
-            L.scales = base.scales.clone()
-            L.ws = q.workspace(M, base.K, base.N)
-            layers.append(L)
-        fn = lambda i: layers[i % R].call(q)  # noqa: E731
-        n = 400 if M <= 64 else 100
-        for g in run_steps(fn, 10, 10):
-            g.replay()
-        secs, _, _ = time_graphs(run_steps(fn, n, 50), ws)
-        secs = max_over_ranks(secs, ws)
-        us = secs / n * 1e6
-        out[str(M)] = {"path": q.qgemm_path_for(M, base.K, base.N), "us": round(us, 2),
-                       "gbs": round(one / us / 1e3, 1),
-                       "tflops": round(2.0 * M * base.K * base.N / us / 1e6, 2)}
-        del layers, base
+        rot, tuned = rotation(q, w, M)
+        R = len(rot)
+        c = R * max(1, math.ceil(8 / R))
+        st = iqm_time(lambda i: rot[i % R].call(q), c, ws, min_replays=100 if M <= 64 else 40,
+                      min_secs=0.1, warm_replays=5)
+        L = rot[0]
+        nbytes, flops = L.nbytes(), 2.0 * M * L.K * L.N
+        out[str(M)] = {"path": q.qgemm_path_for(M, L.K, L.N), "tuned": tuned, "us": round(st["secs"] * 1e6, 2),
+                       "gbs": round(nbytes / st["secs"] / 1e9, 1),
+                       "tflops": round(flops / st["secs"] / 1e12, 2),
+                       "roofline": mixed_roofline(nbytes, flops, st["secs"], pk)}
+        del rot, L
         torch.cuda.empty_cache()
     return out
 
 
-def bench_stack(q, w, steps, ws):
-    """The 80-layer linear stack at M = 1: tokens/s = 1 / (time of all calls)."""
+def bench_stack(q, w, pk, ws):
+    """The 80-layer linear stack at M = 1: tokens/s = 1 / (time of all calls
+    of one token), IQM over token replays."""
     calls = []
     for layer in range(w.layers):
         for mi in range(len(w.matrices)):
             calls.append(Layer(w, 1, layer=layer, matrix=mi))
-    total_bytes = sum(call_bytes(c.K, c.N, 1, c.rows) for c in calls)
-    fn = lambda i: calls[i % len(calls)].call(q)  # noqa: E731
-    n = len(calls) * steps
-    for g in run_steps(fn, len(calls), len(calls)):
-        g.replay()
-    secs, _, _ = time_graphs(run_steps(fn, n, len(calls)), ws)
-    secs = max_over_ranks(secs, ws)
-    tok_s = steps / secs
-    out = {"tokens_per_s": round(tok_s, 2), "calls_per_token": len(calls),
-           "bytes_per_token": total_bytes, "gbs": round(total_bytes * tok_s / 1e9, 1)}
+    n = len(calls)
+    tuned = {f"{c.K}x{c.N}": tune(q, c) for c in calls[:len(w.matrices)]}   # one call per shape
+    total_bytes = sum(c.nbytes() for c in calls)
+    st = iqm_time(lambda i: calls[i % n].call(q), n, ws, min_replays=20, min_secs=0.3, warm_replays=3)
+    tok_s = 1.0 / (st["secs"] * n)
+    roof = pk["hbm"] * 1e9 / total_bytes
+    out = {"tokens_per_s": round(tok_s, 2), "unit": "tokens/s", "calls_per_token": n,
+           "bytes_per_token": total_bytes, "gbs": round(total_bytes * tok_s / 1e9, 1),
+           "replays": st["replays"], "tuned": tuned,
+           "roofline": {"bound": "hbm", "achieved": round(tok_s, 2), "peak": round(roof, 2),
+                        "unit": "tokens/s", "frac": round(tok_s / roof, 4),
+                        "peak_source": pk["src"] + " HBM GB/s / bytes per token"}}
     del calls
     torch.cuda.empty_cache()
     return out
 
 
-def bench_e2e(q, L, steps, warmup, ws):
-    """Public call with host buffers: x in from pinned memory, y back, every step."""
-    xh = L.x.cpu().pin_memory()
-    yh = torch.empty(L.y.shape, dtype=L.y.dtype).pin_memory()
-    xd = torch.empty_like(L.x)
+def bench_e2e(q, rot, steps, warmup, ws):
+    """Public call with host buffers: x in from pinned memory, y back, every
+    step, over the same rotated weight copies as the device-timed leg."""
+    L0 = rot[0]
+    R = len(rot)
+    xh = L0.x.cpu().pin_memory()
+    yh = torch.empty(L0.y.shape, dtype=L0.y.dtype).pin_memory()
+    xd = torch.empty_like(L0.x)
 
-    def step():
+    def step(i):
         xd.copy_(xh, non_blocking=True)
-        L.call(q, x=xd)
-        yh.copy_(L.y, non_blocking=True)
+        rot[i % R].call(q, x=xd)
+        yh.copy_(L0.y, non_blocking=True)
 
-    for _ in range(max(3, min(warmup, 50))):
-        step()
-    n = max(1, min(steps, 2000))
+    for i in range(max(3, min(warmup, 50))):
+        step(i)
+    n = max(1, min(steps, 4000))
     torch.cuda.synchronize()
     barrier(ws)
     t0 = time.perf_counter()
-    for _ in range(n):
-        step()
+    for i in range(n):
+        step(i)
     torch.cuda.synchronize()
     secs = max_over_ranks(time.perf_counter() - t0, ws)
-    return dict(gbs=L_bytes(L) * n / secs / 1e9, steps=n, h2d=xh.numel() * xh.element_size(),
+    return dict(gbs=L0.nbytes() * n / secs / 1e9, steps=n, h2d=xh.numel() * xh.element_size(),
                 d2h=yh.numel() * yh.element_size())
-
-
-def L_bytes(L):
-    return call_bytes(L.K, L.N, L.M, L.rows)
 
 
 def cpu_baseline(w, M):
@@ -433,28 +538,30 @@ def run_ours(args):
     ws, rank, local = dist_setup(args)
     import mixed_bitwidth_weight_b200 as q
     w = W.WORKLOADS[HEADLINE]
-    M = 1
     pk = peaks()
     sampler = ClockSampler(local)
-    if rank == 0 or True:
-        sampler.start()
+    sampler.start()
     time.sleep(0.2)
-    res = bench_decode(q, w, M, args.steps, args.warmup, ws)
+    res = bench_headline(q, w, args.steps, args.warmup, ws)
     clocks = sampler.summary(res["t0"], res["t1"])
+    e2e = bench_e2e(q, res["rot"], args.steps, args.warmup, ws)
+    res.pop("rot")
+    torch.cuda.empty_cache()
+
+    tc0 = time.time()
+    configs = {CFG1: bench_decode_leg(q, W.WORKLOADS[CFG1], 1, pk, ws)}
+    configs[HEADLINE] = {str(m): bench_decode_leg(q, w, m, pk, ws) for m in (2, 4, 8)}
     wp = W.WORKLOADS[PREFILL]
-    pre = bench_prefill(q, wp, PREFILL_M, max(16, min(160, args.steps // 100)), 5, ws)
+    pre = bench_prefill(q, wp, PREFILL_M, pk, ws)
     pre_clocks = sampler.summary(pre["t0"], pre["t1"])
-    extra = {}
-    if args.full:
-        extra["decode_m_gbs"] = {}
-        for m in (2, 4, 8, 16):
-            r = bench_decode(q, w, m, min(args.steps, 2000), min(args.warmup, 200), ws)
-            extra["decode_m_gbs"][str(m)] = round(r["gbs"], 1)
-        extra["crossover_sweep"] = bench_sweep(q, W.WORKLOADS[SWEEP], SWEEP_MS, ws)
-        extra["stack"] = bench_stack(q, W.WORKLOADS[STACK], 3, ws)
-    e2e = bench_e2e(q, res["layer"], args.steps, args.warmup, ws)
+    if not args.no_stack:
+        configs[STACK] = bench_stack(q, W.WORKLOADS[STACK], pk, ws)
+    configs[SWEEP] = bench_sweep(q, W.WORKLOADS[SWEEP], SWEEP_MS, pk, ws)
+    configs_clocks = sampler.summary(tc0, time.time())
     sampler.stop()
-    cpu = cpu_baseline(w, M) if (rank == 0 and ws == 1 and not args.no_cpu) else None
+    cpu = cpu_baseline(w, 1) if (rank == 0 and ws == 1 and not args.no_cpu) else None
+
+    st = res["stats"]
     achieved = res["bytes"] / (res["us"] * 1e-6) / 1e9
     line = {
         "metric": METRIC,
@@ -469,7 +576,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "f16",
         "data": "synthetic (seeded SplitMix64 inputs; random words = uniform codes)",
-        "config": {"workload": HEADLINE, "M": M, "K": w.K, "N": w.N,
+        "config": {"workload": HEADLINE, "M": 1, "K": w.K, "N": w.N,
                    "bpw": round(res["rows"] / (w.K // 32) + 0.125, 4),
                    "weight_copies": res["copies"],
                    "l2": f"inputs larger than L2: {res['copies']} weight copies rotated "
@@ -478,15 +585,24 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
                      "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4),
                      "traffic": traffic_from_profiles("gemv_int_decode_8192x28672_m1"),
-                     "kernel": "qg::gemv_int_kernel<1> (+ qg::xprep_int_kernel, overlapped by PDL; "
-                               "achieved uses the whole step time)", "peak_source": pk["src"],
+                     "kernel": "the tuned variant's main kernel (qg::gemv_int_kernel<1> for the integer "
+                               "GEMV) + its activation prep, overlapped by PDL; achieved uses the whole "
+                               "step time", "peak_source": pk["src"],
                      "bytes_per_launch": res["bytes"]},
+        "tuned": res["tuned"],
+        "stats": {"statistic": "IQM of per-replay times (5/16 to 11/16 quantiles)",
+                  "us": round(st["secs"] * 1e6, 3), "gbs": round(res["bytes"] / st["secs"] / 1e9, 1),
+                  "frac": round(res["bytes"] / st["secs"] / 1e9 / pk["hbm"], 4),
+                  "replays": st["replays"], "calls_per_replay": st["calls_per_replay"],
+                  "timed_secs": st["timed_secs"]},
+        "configs": configs,
         "prefill": {
             "workload": PREFILL, "M": PREFILL_M, "K": wp.K, "N": wp.N,
             "bpw": round(pre["rows"] / (wp.K // 32) + 0.125, 4), "x_dtype": "bf16",
             "mma_dtype": "f16 (x scaled per row by a power of two, exact)",
             "value": round(pre["tflops"] * ws, 2), "unit": "TFLOP/s", "ms_per_call": round(pre["ms"], 4),
-            "weight_copies": pre["copies"],
+            "weight_copies": pre["copies"], "replays": pre["replays"], "tuned": pre["tuned"],
+            "statistic": "IQM of per-replay times (5/16 to 11/16 quantiles)",
             "roofline": {"bound": "tensor", "achieved": round(pre["tflops"], 1), "peak": pk["bf16"],
                          "unit": "TFLOP/s", "frac": round(pre["tflops"] / pk["bf16"], 4),
                          "peak_sustained": pk["bf16_sust"],
@@ -499,12 +615,15 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e["gbs"] * ws, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                "steps": e2e["steps"], "how": "eager qgemm() per step; x H2D from pinned, y D2H to pinned"},
+                "steps": e2e["steps"],
+                "how": "eager qgemm() per step over the rotated weight copies; x H2D from pinned, "
+                       "y D2H to pinned; wall clock around all steps"},
         "gpu_launches": 2 * args.steps,
-        "gpu_launches_how": "timed decode region: xprep_int_kernel + gemv_int_kernel per step",
+        "gpu_launches_how": "timed decode region: two kernels per step (activation prep + the "
+                            "tuned variant's main kernel)",
         "clocks": clocks,
+        "configs_clocks": configs_clocks,
     }
-    line.update(extra)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:
@@ -581,7 +700,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=2000)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--full", action="store_true", help="also sweep M and the 80-layer stack")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 80-layer stack (21 GB of weights)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
                     help="run a few untimed calls of one leg (for ncu) and exit")

@@ -123,7 +123,83 @@ int qgemm_path_for(int M, int K, int N);
  * memory bytes, out[5] = SM count used.  Host only; returns a qgemm_status. */
 int qgemm_plan_info(int M, int K, int N, int64_t qw_rows, int64_t* out);
 
+/* ------------------------------------------------------------ autotuning
+ * Per-shape choice of the kernel variant, after the runtime autotuning of the
+ * EXL2 kernels (nightvoyager.top exllamav2 report, "创新之处" and "关键设计决策":
+ * each (M, K, N) is timed once, 20 warm-up and 200 timed runs ranked by an
+ * interquartile mean, and the choice cached with the built-in heuristic as
+ * the fallback).  A variant is a kernel family (as qgemm_path_for) and one
+ * knob: the integer GEMV's CTAs per SM (1 or 2), none for the tensor-core
+ * GEMV (0), the GEMM's largest k split (1, 2 or 4).  Candidates for M rows:
+ * the integer GEMV (M <= 4), the tensor-core GEMV (M <= 16), the GEMM (any M).
+ * Choices are kept per (current device, M, K, N) for the life of the process;
+ * qgemm(), qgemm_path_for, qgemm_plan_info and qgemm_workspace_bytes consult
+ * them (the workspace size covers every candidate of M, so any choice fits).
+ * Host state is guarded by a mutex; the choice of a shape can change results
+ * in the last bits (another kernel or split), never beyond the tolerance. */
+
+/* Times every candidate on these operands on `stream` (warmup untimed calls,
+ * then iters calls with an event between consecutive calls; the result in
+ * d_y is the last call's, a correct product), ranks them by the mean of the
+ * per-call times between the 5/16 and 11/16 quantiles and records the
+ * fastest.  Candidates whose workspace exceeds ws_bytes are skipped.
+ * Synchronises `stream`.  Refuses (QGEMM_ERR_UNSUPPORTED) a stream that is
+ * being captured: timing needs a live stream.
+ *   h_results  optional host array of 3 * max_results int64: per candidate
+ *              {path, knob, IQM time in ns, or -1 if skipped};
+ * Returns the number of rows written (>= 0) or a negative qgemm_status
+ * (QGEMM_ERR_WORKSPACE when no candidate fits the workspace). */
+int qgemm_autotune(const void* d_x, int x_dtype, const int32_t* d_perm, const uint32_t* d_qw, int64_t qw_rows,
+                   const uint16_t* d_scales, const uint8_t* d_bits, const int32_t* d_offs, int M, int K, int N,
+                   uint16_t* d_y, void* d_ws, size_t ws_bytes, int warmup, int iters, void* stream,
+                   int64_t* h_results, int max_results);
+
+/* mode 1: qgemm() runs qgemm_autotune (20 warm-up, 200 timed calls) on the
+ * first call of a shape without a recorded choice, unless its stream is being
+ * captured (the built-in choice is used then, and tuning waits for an eager
+ * call); mode 0 (default): never.  Host only. */
+int qgemm_set_autotune(int mode);
+
+/* The recorded choice for (M, K, N) on the current device: returns 1 and
+ * writes *h_path, *h_knob; 0 when there is none.  Host only. */
+int qgemm_tune_lookup(int M, int K, int N, int* h_path, int* h_knob);
+
+/* Records a choice without timing (a caller's saved table, or tests);
+ * QGEMM_ERR_UNSUPPORTED for a variant that cannot serve M rows.  Host only. */
+int qgemm_tune_record(int M, int K, int N, int path, int knob);
+
+/* Forgets every recorded choice.  Host only. */
+int qgemm_tune_clear(void);
+
+/* The ranking statistic: mean of h_values[0..n) sorted, from index
+ * floor(5n/16) to ceil(11n/16) (at least one value); -1 for n <= 0. */
+double qgemm_iqm(const float* h_values, int n);
+
 /* ----------------------------------------------------------- device calls */
+
+/* Quantise fp16 weights into codes and fp16 scales, the step before
+ * qgemm_pack (nightvoyager.top exllamav2 report, "关键设计决策": the adaptive
+ * scale with a 4-bit second-level quantisation of the group scale and a scan
+ * of 96 candidate factors per layer keeping the lowest squared error).
+ * This library's reading of the method, per column n:
+ *   base[g] = max over the blocks j of group g of max |W[k][n]| / 2^(b_j-1);
+ *   qmax = max_g base[g];  qs[g] = clamp(rint(sqrt(base[g] / qmax) * 16), 1, 16);
+ *   candidate i = 0..95: p = (32 + i) / 96, s[g] = fp16(p * (qmax * qs[g]^2 / 256)),
+ *   q = clamp(rint(W * (1 / s)) + 2^(b-1), 0, 2^b - 1) (zero point where s = 0);
+ *   E(i) = sum over columns (in order) of the sum over rows (in order) of
+ *   (W - (q - 2^(b-1)) s)^2 in double; the smallest E wins, the lowest i on ties.
+ * Single precision with each operation rounded to nearest even decides the
+ * codes; the result is bit-exact against any implementation of the same steps.
+ *   d_w      [K][N] fp16 weights, act-order rows (as qgemm_pack's codes);
+ *   d_bits   [K/32] widths;
+ *   d_codes  [K][N] uint8 out, feed to qgemm_pack;  d_scales [ceil(K/128)][N] fp16 out;
+ *   d_err    optional double [96] out: E(i);  d_best optional int32 [1] out: the i kept;
+ *   d_ws     qgemm_quantize_workspace_bytes(K, N) bytes (need not be zeroed).
+ * Widths outside {2,3,4,5,6,8} set QGEMM_DEV_BAD_SCHEDULE.  Finite weights only. */
+size_t qgemm_quantize_workspace_bytes(int K, int N);
+int qgemm_quantize(const uint16_t* d_w, const uint8_t* d_bits, int K, int N, uint8_t* d_codes,
+                   uint16_t* d_scales, double* d_err, int32_t* d_best, void* d_ws, size_t ws_bytes,
+                   void* stream);
 
 /* Pack codes into the layout above.
  *   d_codes [K][N] uint8, row k = act-order row, value < 2^b_j (higher bits of a
@@ -171,8 +247,9 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
  * allowed to allocate behind its host's back, or a latency-bound decode loop
  * that cannot afford cudaMalloc/cudaFree (cudaFree synchronises the device).
  *
- * qgemm_decode_noalloc computes exactly what qgemm() computes for M <= 4 (the
- * integer decode GEMV, same kernels and same split, so the same result) but
+ * qgemm_decode_noalloc computes exactly what qgemm() computes for M <= 4 with
+ * the built-in choice or a tuned integer-GEMV variant (the integer decode
+ * GEMV, same kernels and same split, so the same result) but
  * takes its scratch from a buffer of QGEMM_NOALLOC_SCRATCH_BYTES built into
  * the library.  Every GPU that loads the library holds that buffer until the
  * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no
@@ -180,8 +257,9 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
  *
  *   Arguments, layouts and ownership as qgemm(), without d_ws / ws_bytes.
  *   Limits: 1 <= M <= 4 (QGEMM_ERR_SHAPE otherwise); a shape whose scratch
- *     (qgemm_workspace_bytes(M, K, N)) exceeds QGEMM_NOALLOC_SCRATCH_BYTES is
- *     refused with QGEMM_ERR_WORKSPACE before anything is launched.
+ *     (qgemm_noalloc_scratch_bytes(M, K, N)) exceeds
+ *     QGEMM_NOALLOC_SCRATCH_BYTES is refused with QGEMM_ERR_WORKSPACE before
+ *     anything is launched.
  *   First call on a device: looks up the buffer's device address
  *     (cudaGetSymbolAddress, with that device current) and sets the kernels'
  *     shared-memory attributes; make this first call before any stream
@@ -193,6 +271,10 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
  *     buffer and give wrong results: order them, e.g. on one stream.
  *   Returns a qgemm_status as qgemm(). */
 #define QGEMM_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* Scratch bytes qgemm_decode_noalloc needs for this shape (the integer GEMV's
+ * workspace), 0 when M is outside 1..4 or the shape is invalid.  Host only. */
+size_t qgemm_noalloc_scratch_bytes(int M, int K, int N);
 
 int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm,
                          const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scales,

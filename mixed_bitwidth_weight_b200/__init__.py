@@ -8,7 +8,9 @@ package fails if ``libqgemm.so`` has not been built (``build()``).
 
 Names follow the C entry points: ``qgemm_pack``, ``qgemm_dequant``, ``qgemm``,
 ``qgemm_workspace_bytes``, ``qgemm_packed_word_rows``, ``qgemm_offsets``,
-``qgemm_validate_schedule``, ``qgemm_device_error``, ``qgemm_path_for``.
+``qgemm_validate_schedule``, ``qgemm_device_error``, ``qgemm_path_for``,
+``qgemm_autotune``, ``qgemm_set_autotune``, ``qgemm_tune_lookup``,
+``qgemm_tune_record``, ``qgemm_tune_clear``, ``qgemm_iqm``, ``qgemm_quantize``.
 """
 from __future__ import annotations
 
@@ -55,6 +57,15 @@ def _load():
         "qgemm_dequant": (I, [P, I64, P, P, P, I, I, P, P]),
         "qgemm": (I, [P, I, P, P, I64, P, P, P, I, I, I, P, P, SZ, P]),
         "qgemm_decode_noalloc": (I, [P, I, P, P, I64, P, P, P, I, I, I, P, P]),
+        "qgemm_autotune": (I, [P, I, P, P, I64, P, P, P, I, I, I, P, P, SZ, I, I, P, P, I]),
+        "qgemm_set_autotune": (I, [I]),
+        "qgemm_noalloc_scratch_bytes": (SZ, [I, I, I]),
+        "qgemm_quantize_workspace_bytes": (SZ, [I, I]),
+        "qgemm_quantize": (I, [P, P, I, I, P, P, P, P, P, SZ, P]),
+        "qgemm_tune_lookup": (I, [I, I, I, P, P]),
+        "qgemm_tune_record": (I, [I, I, I, I, I]),
+        "qgemm_tune_clear": (I, []),
+        "qgemm_iqm": (ctypes.c_double, [P, I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -181,6 +192,37 @@ def qgemm_plan_info(M: int, K: int, N: int, qw_rows: int) -> dict:
     return dict(path=out[0], grid=out[1], ring=out[2], ctas_per_sm=out[3], smem=out[4], sms=out[5])
 
 
+PATH_NAMES = {0: "integer GEMV", 1: "tensor-core GEMV", 2: "GEMM"}
+
+
+def qgemm_set_autotune(mode: int) -> None:
+    """1: qgemm() tunes each new shape on its first eager call; 0: never."""
+    _ok(_lib.qgemm_set_autotune(int(mode)), "qgemm_set_autotune")
+
+
+def qgemm_tune_lookup(M: int, K: int, N: int):
+    """The recorded (path, knob) for this shape on the current device, or None."""
+    path, knob = ctypes.c_int(0), ctypes.c_int(0)
+    found = _ok(_lib.qgemm_tune_lookup(M, K, N, ctypes.byref(path), ctypes.byref(knob)), "qgemm_tune_lookup")
+    return (path.value, knob.value) if found else None
+
+
+def qgemm_tune_record(M: int, K: int, N: int, path: int, knob: int) -> None:
+    _ok(_lib.qgemm_tune_record(M, K, N, int(path), int(knob)), "qgemm_tune_record")
+
+
+def qgemm_tune_clear() -> None:
+    _ok(_lib.qgemm_tune_clear(), "qgemm_tune_clear")
+
+
+def qgemm_iqm(values) -> float:
+    v = np.ascontiguousarray(np.asarray(values, dtype=np.float32))
+    r = _lib.qgemm_iqm(ctypes.c_void_p(v.ctypes.data), int(v.size))
+    if r < 0:
+        raise ValueError("qgemm_iqm needs at least one value")
+    return float(r)
+
+
 def qgemm_device_error(clear: bool = True) -> int:
     code = ctypes.c_int(0)
     _ok(_lib.qgemm_device_error(ctypes.byref(code), 1 if clear else 0), "qgemm_device_error")
@@ -226,6 +268,37 @@ def qgemm_dequant(qw, scales, bits, offs, w, stream=None):
     return w
 
 
+def qgemm_quantize(w, bits, codes, scales, err=None, best=None, ws=None, stream=None):
+    """fp16 W [K, N] (act-order rows) -> codes uint8 [K, N] and fp16 scales
+    [ceil(K/128), N]; err (float64 [96]) and best (int32 [1]) optional."""
+    import torch
+    if w.dim() != 2 or codes.dim() != 2 or tuple(codes.shape) != tuple(w.shape):
+        _shape_error("w and codes must both be [K, N]")
+    K, N = w.shape
+    if K % 32 != 0:
+        _shape_error(f"K = {K} is not a multiple of 32")
+    if bits.numel() != K // 32:
+        _shape_error(f"bits has {bits.numel()} entries, K/32 = {K // 32} expected")
+    G = (K + 127) // 128
+    if scales.numel() != G * N or (scales.dim() == 2 and tuple(scales.shape) != (G, N)):
+        _shape_error(f"scales must be [ceil(K/128) = {G}, N = {N}], got {tuple(scales.shape)}")
+    if err is not None and err.numel() != 96:
+        _shape_error("err must hold 96 values")
+    if best is not None and best.numel() != 1:
+        _shape_error("best must hold one value")
+    extra = tuple(t for t in (err, best, ws) if t is not None)
+    _check_same_device(w, bits, codes, scales, *extra)
+    if ws is None:
+        ws = torch.empty(max(16, int(_lib.qgemm_quantize_workspace_bytes(K, N))), dtype=torch.uint8,
+                         device=w.device)
+    _ok(_lib.qgemm_quantize(_dev(w, torch.float16, "w"), _dev(bits, torch.uint8, "bits"), K, N,
+                            _dev(codes, torch.uint8, "codes"), _dev(scales, torch.float16, "scales"),
+                            ctypes.c_void_p(0) if err is None else _dev(err, torch.float64, "err"),
+                            ctypes.c_void_p(0) if best is None else _dev(best, torch.int32, "best"),
+                            _dev(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "qgemm_quantize")
+    return codes, scales
+
+
 def qgemm(x, perm, qw, scales, bits, offs, y, ws=None, stream=None):
     """y [M, N] fp16 = x[:, perm] . dequant(qw); x fp16 or bf16 [M, K]."""
     import torch
@@ -251,7 +324,39 @@ def qgemm(x, perm, qw, scales, bits, offs, y, ws=None, stream=None):
     return y
 
 
+def qgemm_autotune(x, perm, qw, scales, bits, offs, y, ws, warmup=20, iters=200, stream=None):
+    """Time every kernel variant of this shape on these operands and record
+    the fastest (see include/qgemm.h).  Returns one dict per candidate
+    (path, knob, us: IQM per call or None when skipped) and the chosen one."""
+    import torch
+    _check_qgemm_shapes(x, perm, qw, scales, bits, offs, y)
+    _check_same_device(x, perm, qw, scales, bits, offs, y, ws)
+    M, K = x.shape
+    N = y.shape[1]
+    if x.dtype == torch.float16:
+        xdt = QGEMM_F16
+    elif x.dtype == torch.bfloat16:
+        xdt = QGEMM_BF16
+    else:
+        raise TypeError("x must be float16 or bfloat16")
+    rows = (ctypes.c_int64 * (3 * 16))()
+    n = _ok(_lib.qgemm_autotune(_dev(x, None, "x"), xdt, _dev(perm, torch.int32, "perm"),
+                                _dev(qw, (torch.int32, torch.uint32), "qw"), qw.shape[0],
+                                _dev(scales, torch.float16, "scales"), _dev(bits, torch.uint8, "bits"),
+                                _dev(offs, torch.int32, "offs"), M, K, N, _dev(y, torch.float16, "y"),
+                                _dev(ws, torch.uint8, "ws"), ws.numel(), int(warmup), int(iters),
+                                _stream(stream), rows, 16), "qgemm_autotune")
+    cands = [dict(path=int(rows[3 * i]), knob=int(rows[3 * i + 1]),
+                  us=(rows[3 * i + 2] / 1e3 if rows[3 * i + 2] >= 0 else None)) for i in range(n)]
+    chosen = qgemm_tune_lookup(M, K, N)
+    return dict(candidates=cands, path=chosen[0], knob=chosen[1])
+
+
 NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def qgemm_noalloc_scratch_bytes(M: int, K: int, N: int) -> int:
+    return int(_lib.qgemm_noalloc_scratch_bytes(M, K, N))
 
 
 def qgemm_decode_noalloc(x, perm, qw, scales, bits, offs, y, stream=None):

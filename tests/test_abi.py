@@ -208,4 +208,4 @@ def test_noalloc_scratch_size_agrees_and_serves_every_decode_shape():
     assert m, "header constant not found"
     assert int(m.group(1)) << int(m.group(2)) == q.NOALLOC_SCRATCH_BYTES
     for M in (1, 2, 3, 4):
-        assert q.qgemm_workspace_bytes(M, 65536, 1 << 24) <= q.NOALLOC_SCRATCH_BYTES
+        assert 0 < q.qgemm_noalloc_scratch_bytes(M, 65536, 1 << 24) <= q.NOALLOC_SCRATCH_BYTES

@@ -112,4 +112,4 @@ def test_noalloc_refuses_what_it_cannot_serve(q):
     with pytest.raises(q.QGemmError, match="unsupported shape"):
         q.qgemm_decode_noalloc(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y)
     # the largest decode shape the library accepts still fits the built-in buffer
-    assert q.qgemm_workspace_bytes(4, 65536, 1 << 24) <= q.NOALLOC_SCRATCH_BYTES
+    assert 0 < q.qgemm_noalloc_scratch_bytes(4, 65536, 1 << 24) <= q.NOALLOC_SCRATCH_BYTES
