@@ -18,6 +18,8 @@ Functions (all numpy in, numpy out):
       y = x[:, perm] . dequant(qw), double [M, N] (or [M, len(cols)])
 * ``quantize(w, bits, threads=0)``  fp16 W [K, N] -> codes, fp16 scales, the
       chosen candidate, the 96 candidate errors and the per-column errors
+* ``kv_quantize(v, b)`` / ``kv_dequantize(codes, scales, D, b)``  Hadamard-
+      rotated KV-cache vectors [n, D] <-> packed codes [n, D/32, b] + scales
 
 Parity pins for every function are in ``tests/test_oracle.py``.
 """
@@ -74,6 +76,10 @@ def _bind(lib):
                                      P, ctypes.c_int64, P, ctypes.c_int]
     lib.oracle_quantize.restype = ctypes.c_int
     lib.oracle_quantize.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P, P, P, P, ctypes.c_int]
+    lib.oracle_kv_quantize.restype = ctypes.c_int
+    lib.oracle_kv_quantize.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P]
+    lib.oracle_kv_dequantize.restype = ctypes.c_int
+    lib.oracle_kv_dequantize.argtypes = [P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P]
     lib.oracle_half_to_double_n.restype = None
     lib.oracle_half_to_double_n.argtypes = [P, P, ctypes.c_int64]
     lib.oracle_double_to_half_n.restype = None
@@ -215,6 +221,25 @@ class Oracle:
                                                _ptr(colerr), _ptr(err), threads), "quantize")
         return Quantized(codes, scales, best, err, colerr)
 
+    def kv_quantize(self, v, b: int):
+        """fp16 vectors [n, D] -> (codes uint32 [n, D/32, b], scales fp16 bits [n, D/32])."""
+        va = np.asarray(v)
+        vb = _c(va.view(np.uint16) if va.dtype == np.float16 else va, np.uint16)
+        n, D = vb.shape
+        codes = np.empty((n, D // 32, b), dtype=np.uint32)
+        scales = np.empty((n, D // 32), dtype=np.uint16)
+        _check(self.lib.oracle_kv_quantize(_ptr(vb), n, D, b, _ptr(codes), _ptr(scales)), "kv_quantize")
+        return codes, scales
+
+    def kv_dequantize(self, codes, scales, D: int, b: int):
+        """-> fp16 bit patterns [n, D]."""
+        c = _c(codes, np.uint32)
+        s = self._scales_bits(scales)
+        n = s.shape[0]
+        out = np.empty((n, D), dtype=np.uint16)
+        _check(self.lib.oracle_kv_dequantize(_ptr(c), _ptr(s), n, D, b, _ptr(out)), "kv_dequantize")
+        return out
+
 
 class Quantized:
     """Result of the oracle's quantiser."""
@@ -268,6 +293,14 @@ def dequant_f16(qw, scales, bits, K):
 
 def quantize(w, bits, threads=0):
     return get().quantize(w, bits, threads)
+
+
+def kv_quantize(v, b):
+    return get().kv_quantize(v, b)
+
+
+def kv_dequantize(codes, scales, D, b):
+    return get().kv_dequantize(codes, scales, D, b)
 
 
 def qgemm_f64(x, perm, qw, scales, bits, cols=None, threads=0):

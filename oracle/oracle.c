@@ -433,3 +433,102 @@ int oracle_quantize(const uint16_t *w, const uint8_t *bits, int K, int N, uint8_
     if (!colerr) free(ce);
     return best;
 }
+
+/* ---------------------------------------------------------------------------
+ * KV-cache quantisation with a Hadamard rotation (nightvoyager.top exllamav2
+ * report, "创新之处": K/V are rotated by a Sylvester/Paley Hadamard matrix and
+ * then quantised to 4 bits; navi2ai ExLlamaV3 page, "核心能力": 2-8 bit caches).
+ * Readings taken here (the pages give no more):
+ *   - each (token, head) vector v of length D (a power of two, 32..256) is
+ *     rotated by the Sylvester matrix H_D (H_1 = [1], H_2n = [[H, H], [H, -H]])
+ *     without normalisation: u = H_D v;
+ *   - u is cut into groups of 32; each group gets one fp16 scale
+ *     s = fp16(max|u| / (2^(b-1) - 1)) and codes
+ *     q = clamp(rint(u * (1 / s)) + 2^(b-1), 0, 2^b - 1) (the zero point where
+ *     s is 0), packed as the weights' 32-code blocks (b words, code r at bits
+ *     [r b, r b + b) of the LSB-first stream);
+ *   - dequantisation: u' = (q - 2^(b-1)) s, v' = fp16((H_D u') / D)
+ *     (H_D H_D = D I).
+ * The rotation runs as the fast Walsh-Hadamard transform in single precision,
+ * stage by stage with strides 1, 2, 4, ..., D/2, each stage replacing the pair
+ * (a at i, b at i + stride) with (a + b, a - b), every operation rounded to
+ * nearest even: the order the GPU kernel uses, so that codes are decided on
+ * the same single-precision values.
+ * ------------------------------------------------------------------------- */
+static int kv_dim_ok(int D) { return D == 32 || D == 64 || D == 128 || D == 256; }
+
+static void fwht_f32(float *a, int D) {
+    for (int st = 1; st < D; st <<= 1)
+        for (int i = 0; i < D; ++i)
+            if (!(i & st)) {
+                float x = a[i], y = a[i + st];
+                a[i] = x + y;
+                a[i + st] = x - y;
+            }
+}
+
+/* v: fp16 bits [nvec][D]; codes: uint32 [nvec][D/32][b]; scales: fp16 bits
+ * [nvec][D/32]. */
+int oracle_kv_quantize(const uint16_t *v, int64_t nvec, int D, int b, uint32_t *codes, uint16_t *scales) {
+    if (!kv_dim_ok(D) || nvec < 0) return ORC_ERR_SHAPE;
+    if (!width_allowed(b)) return ORC_ERR_BITS;
+    float u[256];
+    const int z = 1 << (b - 1), ng = D / 32;
+    for (int64_t t = 0; t < nvec; ++t) {
+        for (int i = 0; i < D; ++i) u[i] = half_to_float(v[t * D + i]);
+        fwht_f32(u, D);
+        for (int g = 0; g < ng; ++g) {
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(u[32 * g + i]);
+                if (a > amax) amax = a;
+            }
+            uint16_t sh = oracle_double_to_half((double)(amax / (float)(z - 1)));
+            scales[t * ng + g] = sh;
+            float s = half_to_float(sh);
+            float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
+            uint32_t *w = codes + (t * ng + g) * b;
+            for (int k = 0; k < b; ++k) w[k] = 0u;
+            for (int i = 0; i < 32; ++i) {
+                int q = z;
+                if (s != 0.0f) {
+                    float r = rintf(u[32 * g + i] * inv);
+                    if (r != r) r = 0.0f;
+                    float lo = (float)(-z), hi = (float)(z - 1);
+                    r = r < lo ? lo : (r > hi ? hi : r);
+                    q = (int)r + z;
+                }
+                for (int k = 0; k < b; ++k)
+                    if ((q >> k) & 1) {
+                        int p = i * b + k;
+                        w[p / 32] |= 1u << (p % 32);
+                    }
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+int oracle_kv_dequantize(const uint32_t *codes, const uint16_t *scales, int64_t nvec, int D, int b, uint16_t *v) {
+    if (!kv_dim_ok(D) || nvec < 0) return ORC_ERR_SHAPE;
+    if (!width_allowed(b)) return ORC_ERR_BITS;
+    float u[256];
+    const int z = 1 << (b - 1), ng = D / 32;
+    for (int64_t t = 0; t < nvec; ++t) {
+        for (int g = 0; g < ng; ++g) {
+            const uint32_t *w = codes + (t * ng + g) * b;
+            float s = half_to_float(scales[t * ng + g]);
+            for (int i = 0; i < 32; ++i) {
+                int q = 0;
+                for (int k = 0; k < b; ++k) {
+                    int p = i * b + k;
+                    q |= (int)((w[p / 32] >> (p % 32)) & 1u) << k;
+                }
+                u[32 * g + i] = (float)(q - z) * s;
+            }
+        }
+        fwht_f32(u, D);
+        for (int i = 0; i < D; ++i) v[t * D + i] = oracle_double_to_half((double)(u[i] / (float)D));
+    }
+    return ORC_OK;
+}

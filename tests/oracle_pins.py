@@ -18,7 +18,11 @@ the oracle disagrees with the fact it checks.  The facts are:
   scales, the p = 1 candidate, zero error); its error equals the squared
   distance to the pinned dequantisation of its output; ties round to even;
   an all-zero column gives zero-point codes and zero scales; codes stay
-  within each block's width and scales on the 16-level grid of the chosen p.
+  within each block's width and scales on the 16-level grid of the chosen p;
+* the KV-cache quantiser: dequantisation equals scipy's Sylvester Hadamard
+  matrix applied to the codes' values and divided by D; vectors built on the
+  grid come back as their codes and scales exactly; random vectors come back
+  within the rounding bound of their group scales.
 
 ``tests/test_oracle.py`` runs them on the oracle and on copies of the oracle
 with planted mistakes, which must each fail at least one pin.
@@ -387,6 +391,81 @@ def pin_quantize_ties_between_candidates_take_the_first(o):
     assert r.best == 0 and (r.err == 0).all()
     assert (r.codes == np.repeat(np.left_shift(1, bits - 1), 32)[:, None]).all()
     assert (r.scales == 0).all()
+
+
+# ------------------------------------------------------------- KV cache
+
+def _kv_pack(q, b):
+    """Codes [n, G, 32] -> words [n, G, b], code r at stream bits [r b, r b + b)."""
+    n, G, _ = q.shape
+    w = np.zeros((n, G, b), dtype=np.uint32)
+    for r in range(32):
+        for k in range(b):
+            p = r * b + k
+            w[:, :, p // 32] |= (((q[:, :, r] >> k) & 1).astype(np.uint32) << np.uint32(p % 32))
+    return w
+
+
+def pin_kv_dequant_is_scaled_hadamard(o):
+    import scipy.linalg
+    rng = _rng(31)
+    for D in (32, 64, 128, 256):
+        for b in (2, 4, 8):
+            n, z = 6, 1 << (b - 1)
+            q = rng.integers(0, 1 << b, size=(n, D // 32, 32))
+            s = np.ldexp(1.0, rng.integers(-3, 2, size=(n, D // 32)))          # exact fp16
+            u = ((q - z) * s[:, :, None]).reshape(n, D)
+            want = (u @ scipy.linalg.hadamard(D).T.astype(np.float64)) / D      # exact in double
+            got = o.kv_dequantize(_kv_pack(q, b), s.astype(np.float16), D, b).view(np.float16)
+            assert np.array_equal(got.astype(np.float64), want.astype(np.float16).astype(np.float64)), (D, b)
+
+
+def pin_kv_grid_roundtrip(o):
+    import scipy.linalg
+    rng = _rng(32)
+    for D in (32, 128, 256):
+        for b in (2, 3, 4, 5, 6, 8):
+            n, z = 5, 1 << (b - 1)
+            m = min(z - 1, 3)                             # small codes keep H u exact in fp16
+            q = z + rng.integers(-m, m + 1, size=(n, D // 32, 32))
+            q[:, :, 7] = 2 * z - 1                        # |q - z| reaches z - 1 in every group
+            s = np.repeat(np.ldexp(1.0, rng.integers(-6, 0, size=(n, 1))), D // 32, axis=1)  # one per vector
+            u = ((q - z) * s[:, :, None]).reshape(n, D)
+            v = (u @ scipy.linalg.hadamard(D).T.astype(np.float64)) / D
+            assert np.array_equal(v.astype(np.float16).astype(np.float64), v)  # exactly representable
+            codes, scales = o.kv_quantize(v.astype(np.float16), b)
+            assert np.array_equal(scales, s.astype(np.float16).view(np.uint16)), (D, b)
+            assert np.array_equal(codes, _kv_pack(q, b)), (D, b)
+
+
+def pin_kv_ties_round_to_even(o):
+    import scipy.linalg
+    D, b, z = 32, 4, 8
+    s = 0.125
+    u = np.zeros(D)
+    u[7] = (z - 1) * s                  # fixes the scale at s
+    u[3], u[5], u[9] = 0.5 * s, 2.5 * s, -1.5 * s
+    v = (scipy.linalg.hadamard(D).astype(np.float64) @ u) / D
+    assert np.array_equal(v.astype(np.float16).astype(np.float64), v)
+    codes, scales = o.kv_quantize(v.astype(np.float16)[None, :], b)
+    q = np.full((1, 1, 32), z)
+    q[0, 0, 7], q[0, 0, 3], q[0, 0, 5], q[0, 0, 9] = 2 * z - 1, z, z + 2, z - 2   # ties to even
+    assert scales[0, 0] == np.float16(s).view(np.uint16)
+    assert np.array_equal(codes, _kv_pack(q, b))
+
+
+def pin_kv_error_within_bound(o):
+    rng = _rng(33)
+    D, n = 128, 64
+    v = (rng.standard_normal((n, D)) * np.exp(rng.standard_normal((n, 1)))).astype(np.float16)
+    v[3, 17] = np.float16(200.0)                          # an outlier channel
+    for b in (2, 4, 8):
+        codes, scales = o.kv_quantize(v, b)
+        back = o.kv_dequantize(codes, scales, D, b).view(np.float16).astype(np.float64)
+        s = o.half_to_double(scales)                      # [n, D/32]
+        bound = 32 * s.sum(axis=1) / 2 / D * (1 + 1e-3)   # |H (u - u')| / D <= sum |u - u'| / D
+        err = np.abs(back - v.astype(np.float64))
+        assert (err <= bound[:, None] + np.abs(back) * 2.0 ** -11 + 1e-7).all(), b
 
 
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

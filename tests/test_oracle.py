@@ -66,6 +66,12 @@ MUTANTS = [
     ("q_candidate_grid", "(float)(32 + i) / 96.0f", "(float)(33 + i) / 96.0f", 0),
     ("q_argmin_last_tie", "if (i == 0 || e < best_e) {", "if (i == 0 || e <= best_e) {", 0),
     ("q_clamp_high", "hi = (float)((1 << b) - 1 - z);", "hi = (float)((1 << b) - z);", 0),
+    # the KV-cache quantiser
+    ("kv_butterfly_sign", "a[i + st] = x - y;", "a[i + st] = y - x;", 0),
+    ("kv_no_inverse_scale", "(double)(u[i] / (float)D)", "(double)(u[i])", 0),
+    ("kv_scale_divisor", "(double)(amax / (float)(z - 1))", "(double)(amax / (float)z)", 0),
+    ("kv_round_away", "float r = rintf(u[32 * g + i] * inv);", "float r = roundf(u[32 * g + i] * inv);", 0),
+    ("kv_group_of_32", "float a = fabsf(u[32 * g + i]);", "float a = fabsf(u[i]);", 0),
     ("q_group_of_row", "int g = k / ORC_GROUP;\n        if (g != g_cur) {",
      "int g = k / ORC_BLOCK / 4 % 2;\n        if (g != g_cur) {", 0),
 ]
