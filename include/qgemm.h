@@ -196,6 +196,27 @@ double qgemm_iqm(const float* h_values, int n);
  *   d_err    optional double [96] out: E(i);  d_best optional int32 [1] out: the i kept;
  *   d_ws     qgemm_quantize_workspace_bytes(K, N) bytes (need not be zeroed).
  * Widths outside {2,3,4,5,6,8} set QGEMM_DEV_BAD_SCHEDULE.  Finite weights only. */
+/* KV-cache quantisation with a Hadamard rotation (nightvoyager.top exllamav2
+ * report, "创新之处": rotated K/V in a 4-bit cache; navi2ai ExLlamaV3 page,
+ * "核心能力": 2-8 bit caches).  Each of the nvec (token, head) vectors of
+ * length D (32, 64, 128 or 256) is rotated by the Sylvester Hadamard matrix
+ * (u = H_D v, fast Walsh-Hadamard transform in single precision, strides 1 ..
+ * D/2, each operation rounded to nearest even), cut into groups of 32 with
+ * one fp16 scale s = fp16(max|u| / (2^(b-1) - 1)) each, and rounded to codes
+ * q = clamp(rint(u * (1 / s)) + 2^(b-1), 0, 2^b - 1) (the zero point where
+ * s = 0), packed as the weights' blocks: b uint32 words per group, code r at
+ * bits [r b, r b + b) of the LSB-first stream.  Dequantisation rotates back:
+ * v' = fp16(H_D ((q - 2^(b-1)) s) / D).
+ *   d_v      [nvec][D] fp16 (in for quantise, out for dequantise);
+ *   d_codes  [nvec][D/32][bits] uint32;  d_scales [nvec][D/32] fp16;
+ *   bits     2, 3, 4, 5, 6 or 8 (QGEMM_ERR_BITS otherwise).
+ * Pointers: d_codes 4-byte aligned, the fp16 arrays 2-byte aligned.  Finite
+ * inputs only.  Asynchronous on `stream`; nvec = 0 launches nothing. */
+int qgemm_kv_quantize(const uint16_t* d_v, int64_t nvec, int D, int bits, uint32_t* d_codes,
+                      uint16_t* d_scales, void* stream);
+int qgemm_kv_dequantize(const uint32_t* d_codes, const uint16_t* d_scales, int64_t nvec, int D, int bits,
+                        uint16_t* d_v, void* stream);
+
 size_t qgemm_quantize_workspace_bytes(int K, int N);
 int qgemm_quantize(const uint16_t* d_w, const uint8_t* d_bits, int K, int N, uint8_t* d_codes,
                    uint16_t* d_scales, double* d_err, int32_t* d_best, void* d_ws, size_t ws_bytes,
@@ -264,9 +285,12 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
  *     (cudaGetSymbolAddress, with that device current) and sets the kernels'
  *     shared-memory attributes; make this first call before any stream
  *     capture.
- *   Shared state: every call on a device uses the same buffer.  Each call
- *     first zeroes, on its stream, the part that must start at zero (the
- *     per-tile tickets); the rest is overwritten before it is read.  Calls
+ *   Shared state: every call on a device uses the same buffer.  Its first
+ *     256 KiB hold the per-tile tickets of every shape served; they are zero
+ *     when the library loads and every completed call leaves them at zero, so
+ *     calls need no memset; the rest is overwritten before it is read.  A call
+ *     that gave up on a wait (QGEMM_DEV_TIMEOUT in the device error word) can
+ *     leave tickets behind: qgemm_noalloc_reset() zeroes them again.  Calls
  *     that overlap on the GPU (other streams, other threads) race on the
  *     buffer and give wrong results: order them, e.g. on one stream.
  *   Returns a qgemm_status as qgemm(). */
@@ -275,6 +299,10 @@ int qgemm(const void* d_x, int x_dtype, const int32_t* d_perm,
 /* Scratch bytes qgemm_decode_noalloc needs for this shape (the integer GEMV's
  * workspace), 0 when M is outside 1..4 or the shape is invalid.  Host only. */
 size_t qgemm_noalloc_scratch_bytes(int M, int K, int N);
+
+/* Zeroes the tickets of the built-in buffer on `stream` (after a call that
+ * reported QGEMM_DEV_TIMEOUT).  Allocates nothing. */
+int qgemm_noalloc_reset(void* stream);
 
 int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm,
                          const uint32_t* d_qw, int64_t qw_rows, const uint16_t* d_scales,

@@ -10,7 +10,8 @@ Names follow the C entry points: ``qgemm_pack``, ``qgemm_dequant``, ``qgemm``,
 ``qgemm_workspace_bytes``, ``qgemm_packed_word_rows``, ``qgemm_offsets``,
 ``qgemm_validate_schedule``, ``qgemm_device_error``, ``qgemm_path_for``,
 ``qgemm_autotune``, ``qgemm_set_autotune``, ``qgemm_tune_lookup``,
-``qgemm_tune_record``, ``qgemm_tune_clear``, ``qgemm_iqm``, ``qgemm_quantize``.
+``qgemm_tune_record``, ``qgemm_tune_clear``, ``qgemm_iqm``, ``qgemm_quantize``,
+``qgemm_kv_quantize``, ``qgemm_kv_dequantize``.
 """
 from __future__ import annotations
 
@@ -60,8 +61,11 @@ def _load():
         "qgemm_autotune": (I, [P, I, P, P, I64, P, P, P, I, I, I, P, P, SZ, I, I, P, P, I]),
         "qgemm_set_autotune": (I, [I]),
         "qgemm_noalloc_scratch_bytes": (SZ, [I, I, I]),
+        "qgemm_noalloc_reset": (I, [P]),
         "qgemm_quantize_workspace_bytes": (SZ, [I, I]),
         "qgemm_quantize": (I, [P, P, I, I, P, P, P, P, P, SZ, P]),
+        "qgemm_kv_quantize": (I, [P, I64, I, I, P, P, P]),
+        "qgemm_kv_dequantize": (I, [P, P, I64, I, I, P, P]),
         "qgemm_tune_lookup": (I, [I, I, I, P, P]),
         "qgemm_tune_record": (I, [I, I, I, I, I]),
         "qgemm_tune_clear": (I, []),
@@ -299,6 +303,43 @@ def qgemm_quantize(w, bits, codes, scales, err=None, best=None, ws=None, stream=
     return codes, scales
 
 
+def _kv_shapes(v, codes, scales, bits):
+    if v.dim() < 1:
+        _shape_error("v must have a last dimension D")
+    D = v.shape[-1]
+    if D not in (32, 64, 128, 256):
+        _shape_error(f"D = {D} must be 32, 64, 128 or 256")
+    nvec = v.numel() // D
+    if codes.numel() != nvec * (D // 32) * bits:
+        _shape_error(f"codes must hold {nvec} x {D // 32} x {bits} words, got {codes.numel()}")
+    if scales.numel() != nvec * (D // 32):
+        _shape_error(f"scales must hold {nvec} x {D // 32} values, got {scales.numel()}")
+    return nvec, D
+
+
+def qgemm_kv_quantize(v, bits, codes, scales, stream=None):
+    """fp16 vectors v [..., D] -> codes int32/uint32 [..., D/32, bits] and fp16
+    scales [..., D/32] (Hadamard rotation, then b-bit groups of 32)."""
+    import torch
+    nvec, D = _kv_shapes(v, codes, scales, bits)
+    _check_same_device(v, codes, scales)
+    _ok(_lib.qgemm_kv_quantize(_dev(v, torch.float16, "v"), nvec, D, int(bits),
+                               _dev(codes, (torch.int32, torch.uint32), "codes"),
+                               _dev(scales, torch.float16, "scales"), _stream(stream)), "qgemm_kv_quantize")
+    return codes, scales
+
+
+def qgemm_kv_dequantize(codes, scales, bits, v, stream=None):
+    """codes [..., D/32, bits] and fp16 scales -> fp16 vectors v [..., D]."""
+    import torch
+    nvec, D = _kv_shapes(v, codes, scales, bits)
+    _check_same_device(v, codes, scales)
+    _ok(_lib.qgemm_kv_dequantize(_dev(codes, (torch.int32, torch.uint32), "codes"),
+                                 _dev(scales, torch.float16, "scales"), nvec, D, int(bits),
+                                 _dev(v, torch.float16, "v"), _stream(stream)), "qgemm_kv_dequantize")
+    return v
+
+
 def qgemm(x, perm, qw, scales, bits, offs, y, ws=None, stream=None):
     """y [M, N] fp16 = x[:, perm] . dequant(qw); x fp16 or bf16 [M, K]."""
     import torch
@@ -357,6 +398,11 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 
 def qgemm_noalloc_scratch_bytes(M: int, K: int, N: int) -> int:
     return int(_lib.qgemm_noalloc_scratch_bytes(M, K, N))
+
+
+def qgemm_noalloc_reset(stream=None) -> None:
+    """Zero the built-in buffer's tickets (after a QGEMM_DEV_TIMEOUT)."""
+    _ok(_lib.qgemm_noalloc_reset(_stream(stream)), "qgemm_noalloc_reset")
 
 
 def qgemm_decode_noalloc(x, perm, qw, scales, bits, offs, y, stream=None):

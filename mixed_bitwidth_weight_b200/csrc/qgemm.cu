@@ -16,6 +16,7 @@
 #include "gemv_int.cuh"
 #include "gemm.cuh"
 #include "quantize.cuh"
+#include "kv_cache.cuh"
 
 namespace {
 
@@ -306,12 +307,14 @@ struct IntWs {
     size_t tickets, slots, rec, total;
 };
 
-IntWs int_ws_layout(int M, int K, int N, int sms) {
+// min_tickets: a larger leading ticket region (the allocation-free entry
+// point keeps one fixed region for every shape it serves).
+IntWs int_ws_layout(int M, int K, int N, int sms, size_t min_tickets = 0) {
     const int mp = int_mp(M);
     const int nb = K / kBlockRows;
     IntWs w;
     w.tickets = 0;
-    w.slots = ticket_region(M, N);
+    w.slots = std::max(ticket_region(M, N), min_tickets);
     w.rec = w.slots + align_up((size_t)gemv_max_grid(K, N, sms) * 2 * mp * kGemvTileCols * 4, 256);
     w.total = w.rec + align_up((size_t)(nb + 8) * int_rec_bytes(mp), 256);
     return w;
@@ -370,11 +373,12 @@ cudaError_t launch_int(const GemvPlan& plan, const IntParams& p, const IntMaps& 
 
 int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
                  const uint16_t* scales, const uint8_t* bits, const int32_t* offs, int M, int K, int N,
-                 uint16_t* y, void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev, int cps_req = 0) {
+                 uint16_t* y, void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev, int cps_req = 0,
+                 size_t min_tickets = 0) {
     GemvPlan plan;
     int st = plan_int(M, K, N, qw_rows, dev->sms, &plan, nullptr, cps_req);
     if (st != QGEMM_OK) return st;
-    const IntWs L = int_ws_layout(M, K, N, dev->sms);
+    const IntWs L = int_ws_layout(M, K, N, dev->sms, min_tickets);
     if (ws_bytes < L.total || ws == nullptr) return QGEMM_ERR_WORKSPACE;
     int devid = 0;
     if (cudaGetDevice(&devid) != cudaSuccess) return QGEMM_ERR_CUDA;
@@ -597,6 +601,12 @@ int run_gemm(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw
 // host-side stand-in, not device memory: kernels get the address that
 // cudaGetSymbolAddress returns for the current device.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[QGEMM_NOALLOC_SCRATCH_BYTES];
+
+// Its first kNoAllocTickets bytes hold the tickets of every shape served (the
+// largest N accepted has 65536 tiles): no call writes data there, and every
+// completed call leaves its tickets at zero, so the region is zero at every
+// call without a memset (it is zero when the module loads).
+constexpr size_t kNoAllocTickets = (size_t)256 << 10;
 
 void* g_noalloc_ptr[64];
 std::mutex g_noalloc_mu;
@@ -1128,9 +1138,53 @@ int qgemm_quantize(const uint16_t* d_w, const uint8_t* d_bits, int K, int N, uin
     return launch_status();
 }
 
+int qgemm_kv_quantize(const uint16_t* d_v, int64_t nvec, int D, int bits, uint32_t* d_codes, uint16_t* d_scales,
+                      void* stream) {
+    if (!d_v || !d_codes || !d_scales) return QGEMM_ERR_NULL;
+    if (nvec < 0 || nvec > ((int64_t)1 << 36) || (D != 32 && D != 64 && D != 128 && D != 256))
+        return QGEMM_ERR_SHAPE;
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 5 || bits == 6 || bits == 8)) return QGEMM_ERR_BITS;
+    if (((uintptr_t)d_v & 1) || ((uintptr_t)d_codes & 3) || ((uintptr_t)d_scales & 1)) return QGEMM_ERR_ALIGN;
+    if (nvec == 0) return QGEMM_OK;
+    const int64_t per_cta = (int64_t)kKvWarps * kKvPerWarp;
+    const dim3 grid((unsigned)((nvec + per_cta - 1) / per_cta)), block(32 * kKvWarps);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const __half* v = reinterpret_cast<const __half*>(d_v);
+    __half* sc = reinterpret_cast<__half*>(d_scales);
+    switch (D / 32) {
+        case 1: kv_quant_kernel<1><<<grid, block, 0, s>>>(v, nvec, bits, d_codes, sc); break;
+        case 2: kv_quant_kernel<2><<<grid, block, 0, s>>>(v, nvec, bits, d_codes, sc); break;
+        case 4: kv_quant_kernel<4><<<grid, block, 0, s>>>(v, nvec, bits, d_codes, sc); break;
+        default: kv_quant_kernel<8><<<grid, block, 0, s>>>(v, nvec, bits, d_codes, sc); break;
+    }
+    return launch_status();
+}
+
+int qgemm_kv_dequantize(const uint32_t* d_codes, const uint16_t* d_scales, int64_t nvec, int D, int bits,
+                        uint16_t* d_v, void* stream) {
+    if (!d_v || !d_codes || !d_scales) return QGEMM_ERR_NULL;
+    if (nvec < 0 || nvec > ((int64_t)1 << 36) || (D != 32 && D != 64 && D != 128 && D != 256))
+        return QGEMM_ERR_SHAPE;
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 5 || bits == 6 || bits == 8)) return QGEMM_ERR_BITS;
+    if (((uintptr_t)d_v & 1) || ((uintptr_t)d_codes & 3) || ((uintptr_t)d_scales & 1)) return QGEMM_ERR_ALIGN;
+    if (nvec == 0) return QGEMM_OK;
+    const int64_t per_cta = (int64_t)kKvWarps * kKvPerWarp;
+    const dim3 grid((unsigned)((nvec + per_cta - 1) / per_cta)), block(32 * kKvWarps);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    __half* v = reinterpret_cast<__half*>(d_v);
+    const __half* sc = reinterpret_cast<const __half*>(d_scales);
+    switch (D / 32) {
+        case 1: kv_dequant_kernel<1><<<grid, block, 0, s>>>(d_codes, sc, nvec, bits, v); break;
+        case 2: kv_dequant_kernel<2><<<grid, block, 0, s>>>(d_codes, sc, nvec, bits, v); break;
+        case 4: kv_dequant_kernel<4><<<grid, block, 0, s>>>(d_codes, sc, nvec, bits, v); break;
+        default: kv_dequant_kernel<8><<<grid, block, 0, s>>>(d_codes, sc, nvec, bits, v); break;
+    }
+    return launch_status();
+}
+
 size_t qgemm_noalloc_scratch_bytes(int M, int K, int N) {
     if (M < 1 || M > kNoAllocMaxM || check_shape(K, N) != QGEMM_OK) return 0;
-    return int_ws_layout(M, K, N, device_sms()).total;
+    return int_ws_layout(M, K, N, device_sms(), kNoAllocTickets).total;
 }
 
 int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm, const uint32_t* d_qw,
@@ -1146,21 +1200,27 @@ int qgemm_decode_noalloc(const void* d_x, int x_dtype, const int32_t* d_perm, co
         return QGEMM_ERR_ALIGN;
     DeviceInfo* dev = nullptr;
     if ((st = current_device_info(&dev)) != QGEMM_OK) return st;
-    const IntWs L = int_ws_layout(M, K, N, dev->sms);
-    if (L.total > QGEMM_NOALLOC_SCRATCH_BYTES) return QGEMM_ERR_WORKSPACE;
+    const IntWs L = int_ws_layout(M, K, N, dev->sms, kNoAllocTickets);
+    if (L.slots > kNoAllocTickets || L.total > QGEMM_NOALLOC_SCRATCH_BYTES) return QGEMM_ERR_WORKSPACE;
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != QGEMM_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the tickets (the layout's first bytes, up to the partial-sum slots) must start at zero
-    if (cudaMemsetAsync(scratch, 0, L.slots, s) != cudaSuccess) {
-        cudaGetLastError();
-        return QGEMM_ERR_CUDA;
-    }
     // the CTA count qgemm() would use: a tuned integer-GEMV variant, else the built-in one
     Variant v;
     const int cps = (tuned_variant(M, K, N, &v) && v.path == kPathGemvInt) ? v.knob : 0;
     return run_gemv_int(d_x, x_dtype, d_perm, d_qw, qw_rows, d_scales, d_bits, d_offs, M, K, N, d_y, scratch,
-                        QGEMM_NOALLOC_SCRATCH_BYTES, s, dev, cps);
+                        QGEMM_NOALLOC_SCRATCH_BYTES, s, dev, cps, kNoAllocTickets);
+}
+
+int qgemm_noalloc_reset(void* stream) {
+    void* scratch = nullptr;
+    const int st = noalloc_scratch(&scratch);
+    if (st != QGEMM_OK) return st;
+    if (cudaMemsetAsync(scratch, 0, kNoAllocTickets, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return QGEMM_ERR_CUDA;
+    }
+    return QGEMM_OK;
 }
 
 }  // extern "C"

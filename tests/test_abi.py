@@ -209,3 +209,29 @@ def test_noalloc_scratch_size_agrees_and_serves_every_decode_shape():
     assert int(m.group(1)) << int(m.group(2)) == q.NOALLOC_SCRATCH_BYTES
     for M in (1, 2, 3, 4):
         assert 0 < q.qgemm_noalloc_scratch_bytes(M, 65536, 1 << 24) <= q.NOALLOC_SCRATCH_BYTES
+
+
+def test_kv_cache_entry_points_check_arguments_on_the_host():
+    lib = q._lib
+    P = ctypes.c_void_p
+    dummy = P(16)
+    assert lib.qgemm_kv_quantize(None, 1, 128, 4, dummy, dummy, None) == -1       # null
+    assert lib.qgemm_kv_quantize(dummy, 1, 96, 4, dummy, dummy, None) == -2       # D not a power of two
+    assert lib.qgemm_kv_quantize(dummy, -1, 128, 4, dummy, dummy, None) == -2     # negative count
+    assert lib.qgemm_kv_quantize(dummy, 1, 128, 7, dummy, dummy, None) == -3      # width
+    assert lib.qgemm_kv_quantize(P(17), 1, 128, 4, dummy, dummy, None) == -4      # alignment
+    assert lib.qgemm_kv_dequantize(dummy, dummy, 1, 512, 4, dummy, None) == -2
+    assert lib.qgemm_kv_dequantize(dummy, dummy, 1, 128, 1, dummy, None) == -3
+    assert lib.qgemm_kv_quantize(dummy, 0, 128, 4, dummy, dummy, None) == 0       # nothing to do
+
+
+def test_quantize_entry_point_checks_arguments_on_the_host():
+    lib = q._lib
+    P = ctypes.c_void_p
+    d = P(256)
+    ws = q._lib.qgemm_quantize_workspace_bytes(256, 64)
+    assert ws > 0
+    assert lib.qgemm_quantize(None, d, 256, 64, d, d, None, None, d, ws, None) == -1
+    assert lib.qgemm_quantize(d, d, 250, 64, d, d, None, None, d, ws, None) == -2   # K % 32
+    assert lib.qgemm_quantize(d, d, 256, 64, P(264), d, None, None, d, ws, None) == -4
+    assert lib.qgemm_quantize(d, d, 256, 64, d, d, None, None, d, ws - 1, None) == -5

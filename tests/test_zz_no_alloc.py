@@ -113,3 +113,21 @@ def test_noalloc_refuses_what_it_cannot_serve(q):
         q.qgemm_decode_noalloc(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y)
     # the largest decode shape the library accepts still fits the built-in buffer
     assert 0 < q.qgemm_noalloc_scratch_bytes(4, 65536, 1 << 24) <= q.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_reset_then_calls_stay_correct(q):
+    """qgemm_noalloc_reset (the recovery after a call that gave up on a wait)
+    zeroes the tickets; calls before and after it agree with the oracle."""
+    M, K, N = 2, 2048, 1032
+    pr = P.make(K, N, M=M, kind="shuffled", seed=404)
+    g = P.to_gpu(pr)
+    ref = P.ref_y(pr)
+    args = (g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"])
+    y0 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    q.qgemm_decode_noalloc(*args, y0)
+    q.qgemm_noalloc_reset()
+    y1 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    q.qgemm_decode_noalloc(*args, y1)
+    torch.cuda.synchronize()
+    P.check_close(y0, ref)
+    assert torch.equal(y0, y1)
