@@ -25,6 +25,8 @@ Extra objects on the same line:
                   sweep_8192x8192_3p75     M = 1 ... 512 on one 8192^2 layer,
                                            the GEMV/GEMM crossover, with the
                                            path each M dispatches to;
+                  pack_dequant             the format's pack and dequant
+                                           kernels on the headline layer;
   prefill       TFLOP/s of the M = 2048 prefill GEMM (K = 8192, N = 28672,
                 4.0 bpw, bf16 activations) against the dense tensor peak;
   cpu_baseline  the CPU oracle timed on the host cores (rank 0, N = 1);
@@ -329,6 +331,23 @@ def time_region(graphs, ws):
     return ev[0].elapsed_time(ev[-1]) / 1e3, per, t0, t1
 
 
+def timed_batches(region, ws, min_replays, min_secs, max_replays):
+    """Batches of timed replays until there are at least min_replays lasting
+    at least min_secs in all.  region(n) times n replays and returns (secs,
+    per-replay secs, t0, t1).  Every rank takes the same number of regions
+    (each has barriers): the decision to time another batch uses the slowest
+    rank's total."""
+    per, total, t0, t1 = [], 0.0, None, None
+    while len(per) < min_replays or (total < min_secs and len(per) < max_replays):
+        n = max(1, min_replays - len(per)) if len(per) < min_replays else min_replays
+        secs, p, a, b = region(n)
+        t0 = a if t0 is None else t0
+        t1 = b
+        per += p
+        total += max_over_ranks(secs, ws)
+    return per, total, t0, t1
+
+
 def iqm_time(fn, calls_per_replay, ws, min_replays=200, min_secs=0.2, warm_replays=20, max_replays=4000):
     """Seconds per call of fn as the IQM of per-replay times: warm-up
     replays, then batches of timed replays until there are at least
@@ -337,14 +356,8 @@ def iqm_time(fn, calls_per_replay, ws, min_replays=200, min_secs=0.2, warm_repla
     for _ in range(warm_replays):
         g.replay()
     spin_up(g)
-    per, total, t0, t1 = [], 0.0, None, None
-    while len(per) < min_replays or (total < min_secs and len(per) < max_replays):
-        n = max(1, min_replays - len(per)) if len(per) < min_replays else min_replays
-        secs, p, a, b = time_region([g] * n, ws)
-        t0 = a if t0 is None else t0
-        t1 = b
-        per += p
-        total += secs
+    per, total, t0, t1 = timed_batches(lambda n: time_region([g] * n, ws), ws, min_replays, min_secs,
+                                       max_replays)
     per_call = [p / calls_per_replay for p in per]
     v = max_over_ranks(iqm(per_call), ws)
     del g
@@ -464,6 +477,30 @@ def bench_stack(q, w, pk, ws):
     return out
 
 
+def bench_pack_dequant(q, w, pk, ws):
+    """The format's two HBM-bound kernels on the headline layer: pack (codes
+    uint8 [K, N] -> words) and dequant (words + scales -> fp16 W [K, N])."""
+    L = Layer(w, 1, x=False)
+    K, N = L.K, L.N
+    codes = torch.randint(0, 4, (K, N), dtype=torch.uint8, device="cuda")   # < 2^b for every width
+    qw = torch.empty_like(L.qw)
+    wout = torch.empty((K, N), dtype=torch.float16, device="cuda")
+    sp = iqm_time(lambda i: q.qgemm_pack(codes, L.bits, L.offs, qw), 1, ws, min_replays=50, min_secs=0.1,
+                  warm_replays=3)
+    sd = iqm_time(lambda i: q.qgemm_dequant(L.qw, L.scales, L.bits, L.offs, wout), 1, ws, min_replays=50,
+                  min_secs=0.1, warm_replays=3)
+    pb = K * N + 4 * N * L.rows + 4 * (K // 32 + 1) + K // 32
+    db = 4 * N * L.rows + 2 * ((K + 127) // 128) * N + 2 * K * N + 4 * (K // 32 + 1) + K // 32
+    out = {"pack": {"us": round(sp["secs"] * 1e6, 2), "bytes": pb, "gbs": round(pb / sp["secs"] / 1e9, 1),
+                    "roofline": hbm_roofline(pb, sp["secs"], pk["hbm"], pk["src"])},
+           "dequant": {"us": round(sd["secs"] * 1e6, 2), "bytes": db, "gbs": round(db / sd["secs"] / 1e9, 1),
+                       "roofline": hbm_roofline(db, sd["secs"], pk["hbm"], pk["src"])},
+           "shape": f"{K}x{N}, {w.name} schedule"}
+    del L, codes, qw, wout
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_e2e(q, rot, steps, warmup, ws):
     """Public call with host buffers: x in from pinned memory, y back, every
     step, over the same rotated weight copies as the device-timed leg."""
@@ -557,6 +594,7 @@ def run_ours(args):
     if not args.no_stack:
         configs[STACK] = bench_stack(q, W.WORKLOADS[STACK], pk, ws)
     configs[SWEEP] = bench_sweep(q, W.WORKLOADS[SWEEP], SWEEP_MS, pk, ws)
+    configs["pack_dequant"] = bench_pack_dequant(q, w, pk, ws)
     configs_clocks = sampler.summary(tc0, time.time())
     sampler.stop()
     cpu = cpu_baseline(w, 1) if (rank == 0 and ws == 1 and not args.no_cpu) else None

@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tmem_ld16(taddr + c, v);
                 if (nsplit == 1) {
                     if (row < p.M && n0 + c < p.N) store_y(row, c, v, g1, g2);
-                } else {
+                } else if (row < p.M) {  // the reduction reads the tile's rows of x only
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
                         __stcg(reinterpret_cast<float4*>(part + c + 4 * u),

@@ -98,7 +98,7 @@ QG_DEV float quant_bases(const QuantParams& p, int n, const uint8_t* s_bits) {
 }
 
 __global__ void __launch_bounds__(kQuantCols) quant_scan_kernel(const QuantParams p) {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];  // one alignment for every kernel of the library
     double* s_acc = reinterpret_cast<double*>(smem);                          // [96][kQuantCols]
     __half* s_tile = reinterpret_cast<__half*>(s_acc + kQuantCands * kQuantCols);  // [128][kQuantCols]
     uint8_t* s_bits = reinterpret_cast<uint8_t*>(s_tile + 128 * kQuantCols);  // [K/32]
