@@ -144,19 +144,17 @@ QG_DEV constexpr int int_acc_shift(int b) { return b == 2 ? 6 : b == 4 ? 4 : 0; 
 
 // One block of width B for the thread's 4 adjacent columns:
 // acc[q][t] = 2^int_acc_shift(B) * (acc[q][t] + sum_k x_int[t][k] * code[k][col q]).
-// w = word row 0 of the block at the thread's first column.
+// v[i] = word row i of the block at the thread's 4 columns.
 template <int B, int MP>
-QG_DEV void block_dp2a(const uint8_t* w, const uint32_t (&xp)[MP][16], int32_t (&acc)[4][MP]) {
-    auto row = [&](int i) { return *reinterpret_cast<const uint4*>(w + i * kIntRowBytes); };
+QG_DEV void block_dp2a_v(const uint4 (&v)[B], const uint32_t (&xp)[MP][16], int32_t (&acc)[4][MP]) {
     if constexpr (B == 2) {
         // word wi, byte i: codes 16wi+4i+s at bits 2s; mask s keeps q * 4^s
-        const uint4 v0 = row(0), v1 = row(1);
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             const uint32_t mask = 0x03030303u << (2 * s);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint32_t m0 = comp(v0, q) & mask, m1 = comp(v1, q) & mask;
+                const uint32_t m0 = comp(v[0], q) & mask, m1 = comp(v[1], q) & mask;
 #pragma unroll
                 for (int t = 0; t < MP; ++t) {
                     int32_t a = (s == 0) ? acc[q][t] : acc[q][t] * 4;
@@ -169,9 +167,6 @@ QG_DEV void block_dp2a(const uint8_t* w, const uint32_t (&xp)[MP][16], int32_t (
         }
     } else if constexpr (B == 4) {
         // word wi: low nibbles of its bytes are codes 8wi+2i, high nibbles 8wi+2i+1 (as 16 q)
-        uint4 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = row(i);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -195,19 +190,15 @@ QG_DEV void block_dp2a(const uint8_t* w, const uint32_t (&xp)[MP][16], int32_t (
     } else if constexpr (B == 8) {
 #pragma unroll
         for (int wi = 0; wi < 8; ++wi) {
-            const uint4 v = row(wi);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
                 for (int t = 0; t < MP; ++t) {
-                    acc[q][t] = dp2a_lo(xp[t][2 * wi], comp(v, q), acc[q][t]);
-                    acc[q][t] = dp2a_hi(xp[t][2 * wi + 1], comp(v, q), acc[q][t]);
+                    acc[q][t] = dp2a_lo(xp[t][2 * wi], comp(v[wi], q), acc[q][t]);
+                    acc[q][t] = dp2a_hi(xp[t][2 * wi + 1], comp(v[wi], q), acc[q][t]);
                 }
         }
     } else {  // 3, 5, 6: codes 4c..4c+3 from a window at bit 4cB, spread into bytes
-        uint4 v[B];
-#pragma unroll
-        for (int i = 0; i < B; ++i) v[i] = row(i);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
 #pragma unroll
@@ -226,6 +217,16 @@ QG_DEV void block_dp2a(const uint8_t* w, const uint32_t (&xp)[MP][16], int32_t (
             }
         }
     }
+}
+
+// The same, reading the block's word rows from the shared-memory ring (rows
+// kIntRowBytes apart).  w = word row 0 of the block at the thread's first column.
+template <int B, int MP>
+QG_DEV void block_dp2a(const uint8_t* w, const uint32_t (&xp)[MP][16], int32_t (&acc)[4][MP]) {
+    uint4 v[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) v[i] = *reinterpret_cast<const uint4*>(w + i * kIntRowBytes);
+    block_dp2a_v<B, MP>(v, xp, acc);
 }
 
 // ------------------------------------------------------------------ xprep

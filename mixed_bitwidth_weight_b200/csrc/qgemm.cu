@@ -371,6 +371,36 @@ cudaError_t launch_int(const GemvPlan& plan, const IntParams& p, const IntMaps& 
     return cudaLaunchKernelEx(&cfg, gemv_int_kernel<MP>, p, maps);
 }
 
+int launch_xprep_int(const void* x, int x_dtype, const int32_t* perm, const uint8_t* bits, int M, int K,
+                     uint8_t* rec, cudaStream_t stream) {
+    IntPrepParams xp;
+    xp.x = x;
+    xp.perm = perm;
+    xp.bits = bits;
+    xp.rec = rec;
+    xp.M = M;
+    xp.K = K;
+    xp.nb = K / kBlockRows;
+    xp.mp = int_mp(M);
+    xp.x_bf16 = (x_dtype == QGEMM_BF16);
+    // programmatic dependent of the previous grid (it waits for it on the
+    // device), so its launch overlaps that grid's tail
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((xp.nb + 7) / 8);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, xprep_int_kernel, xp) != cudaSuccess) {
+        cudaGetLastError();
+        return QGEMM_ERR_CUDA;
+    }
+    return QGEMM_OK;
+}
+
 int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t* qw, int64_t qw_rows,
                  const uint16_t* scales, const uint8_t* bits, const int32_t* offs, int M, int K, int N,
                  uint16_t* y, void* ws, size_t ws_bytes, cudaStream_t stream, DeviceInfo* dev, int cps_req = 0,
@@ -390,36 +420,10 @@ int run_gemv_int(const void* x, int x_dtype, const int32_t* perm, const uint32_t
     const int nb = K / kBlockRows;
     const int mp = int_mp(M);
 
-    IntPrepParams xp;
-    xp.x = x;
-    xp.perm = perm;
-    xp.bits = bits;
-    xp.rec = w8 + L.rec;
-    xp.M = M;
-    xp.K = K;
-    xp.nb = nb;
-    xp.mp = mp;
-    xp.x_bf16 = (x_dtype == QGEMM_BF16);
-    {
-        // programmatic dependent of the previous grid (it waits for it on the
-        // device), so its launch overlaps that grid's tail
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((nb + 7) / 8);
-        cfg.blockDim = dim3(256);
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, xprep_int_kernel, xp) != cudaSuccess) {
-            cudaGetLastError();
-            return QGEMM_ERR_CUDA;
-        }
-    }
+    if ((st = launch_xprep_int(x, x_dtype, perm, bits, M, K, w8 + L.rec, stream)) != QGEMM_OK) return st;
 
     IntParams p;
-    p.rec = xp.rec;
+    p.rec = w8 + L.rec;
     p.qw = qw;
     p.qw_rows = qw_rows;
     p.scales = reinterpret_cast<const __half*>(scales);
