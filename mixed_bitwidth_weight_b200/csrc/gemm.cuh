@@ -52,6 +52,7 @@ constexpr int kGemmFixedSmem =
 
 struct GemmMaps {
     CUtensorMap a;                    // x_p [M][K], box {64, 256}, 128-byte swizzle
+    CUtensorMap a64;                  // the same with box {64, 64}: tiles with few rows of x
     CUtensorMap w[kGemmBoxMaps];      // qw [qw_rows][N], box {256, 2^i}
 };
 
@@ -308,6 +309,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 0) {
         // ================================================= TMA producer
         if (lane == 0) {
+            const int asub = min(4, (p.M - m0 + 63) / 64);  // 64-row slices of x in this tile
             int i = 0;
             bool ok = true;
             for (; i < nk; ++i) {
@@ -318,8 +320,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 }
                 const int gi = kb + i;  // global k step
-                mbar_arrive_expect_tx(&a_full[sa], (uint32_t)kGemmABytes);
-                tma_load_2d(sA + sa * kGemmABytes, &maps.a, gi * kGemmBK, m0, &a_full[sa]);
+                if (asub == 4) {
+                    mbar_arrive_expect_tx(&a_full[sa], (uint32_t)kGemmABytes);
+                    tma_load_2d(sA + sa * kGemmABytes, &maps.a, gi * kGemmBK, m0, &a_full[sa]);
+                } else {
+                    // only the 64-row slices that hold rows of x; the MMA also
+                    // reads the other rows of the stage, whose accumulator
+                    // rows are never stored
+                    mbar_arrive_expect_tx(&a_full[sa], (uint32_t)(asub * (kGemmABytes / 4)));
+                    for (int q = 0; q < asub; ++q)
+                        tma_load_2d(sA + sa * kGemmABytes + q * (kGemmABytes / 4), &maps.a64, gi * kGemmBK,
+                                    m0 + 64 * q, &a_full[sa]);
+                }
                 const int j0 = 2 * gi, j1 = min(j0 + 2, nb);
                 const int r0 = s_offs[j0], rows = s_offs[j1] - r0;
                 const int g = (gi * kGemmBK) / 128;

@@ -514,6 +514,11 @@ int make_gemm_maps(const void* xp, int x_dtype, int M, int K, const uint32_t* qw
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return QGEMM_ERR_CUDA;
+        const cuuint32_t box64[2] = {(cuuint32_t)kGemmBK, 64u};
+        const CUresult r64 = fn(&maps->a64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(xp), dims, strides,
+                                box64, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r64 != CUDA_SUCCESS) return QGEMM_ERR_CUDA;
     }
     const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)qw_rows};
     const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
