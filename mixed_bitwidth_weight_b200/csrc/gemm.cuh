@@ -8,9 +8,9 @@
 //   both MMA operands are fp16 (bf16 input is scaled per row by a power of
 //   two first, exactly, and y is scaled back).
 // * gemm_kernel computes one 256 x 256 tile of y per CTA.  Warp roles:
-//     warp 0     - TMA producer: activation tiles (256 rows x 64 k, 128-byte
-//                  swizzle) and, per 64-row k step, the step's word rows
-//                  (2D boxes) and its group's scale row;
+//     warp 0     - activation producer: per 64-row k step the activation
+//                  tile (256 rows x 64 k, 128-byte swizzle; only its 64-row
+//                  slices that hold rows of x when there are fewer);
 //     warp 1     - allocates TMEM (two 128 x 256 fp32 accumulators, all 512
 //                  columns) and issues the MMAs from one thread:
 //                  tcgen05.mma kind::f16, M = 128, N = 256, K = 16, both
@@ -21,7 +21,10 @@
 //                  with one rounding (the bit-exact dequantised weight) and
 //                  writes row n of the B tile in the
 //                  K-major 128-byte-swizzled layout the MMA reads; after the
-//                  last step they move the accumulators TMEM -> fp16 y.
+//                  last step they move the accumulators TMEM -> fp16 y;
+//     warp 18    - word-row producer: per k step the step's word rows (2D
+//                  boxes) and its group's scale row (a warp of its own, so
+//                  the two copy streams wait only on their own stages).
 // Every wait is bounded; a timeout sets the device error word, the CTA skips
 // the remaining work, waits for its copies and MMAs and frees TMEM.
 #pragma once
@@ -44,7 +47,8 @@ constexpr int kGemmBBytes = kGemmBN * kGemmBK * 2;       // 32 KB
 constexpr int kGemmRawRows = 16;                         // word rows of two blocks, at most
 constexpr int kGemmRBytes = (kGemmRawRows + 1) * 1024;   // scale row + word rows
 constexpr int kGemmDecWarps = 16;                        // 2 blocks x 256 columns per k step
-constexpr int kGemmThreads = 64 + kGemmDecWarps * 32;
+constexpr int kGemmRawWarp = 2 + kGemmDecWarps;          // the word-row producer (last warp)
+constexpr int kGemmThreads = 64 + kGemmDecWarps * 32 + 32;
 constexpr int kGemmBoxMaps = 5;                          // word boxes of 1, 2, 4, 8, 16 rows
 constexpr int kGemmMaxSplit = 4;                         // k splits of one tile, at most
 constexpr int kGemmFixedSmem =
@@ -307,15 +311,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (s_misc[0]) {
         if (tid == 0) set_dev_error(QGEMM_DEV_BAD_SCHEDULE);
     } else if (warp == 0) {
-        // ================================================= TMA producer
+        // ================================================= activation producer
         if (lane == 0) {
             const int asub = min(4, (p.M - m0 + 63) / 64);  // 64-row slices of x in this tile
             int i = 0;
             bool ok = true;
             for (; i < nk; ++i) {
-                const int sa = i % kGemmAStages, sr = i % kGemmRStages;
-                if ((i >= kGemmAStages && !mbar_wait(&a_empty[sa], (uint32_t)(((i / kGemmAStages) - 1) & 1))) ||
-                    (i >= kGemmRStages && !mbar_wait(&r_empty[sr], (uint32_t)(((i / kGemmRStages) - 1) & 1)))) {
+                const int sa = i % kGemmAStages;
+                if (i >= kGemmAStages && !mbar_wait(&a_empty[sa], (uint32_t)(((i / kGemmAStages) - 1) & 1))) {
                     ok = false;
                     break;
                 }
@@ -332,6 +335,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tma_load_2d(sA + sa * kGemmABytes + q * (kGemmABytes / 4), &maps.a64, gi * kGemmBK,
                                     m0 + 64 * q, &a_full[sa]);
                 }
+            }
+            if (!ok) {  // let every issued copy land before the CTA can exit
+                s_misc[1] = 1;
+                for (int k = max(0, i - kGemmAStages); k < i; ++k)
+                    mbar_wait(&a_full[k % kGemmAStages], (uint32_t)((k / kGemmAStages) & 1));
+            }
+        }
+    } else if (warp == kGemmRawWarp) {
+        // ================================================= word-row producer
+        // (a warp of its own: its copies do not wait behind the activation
+        // tiles' stage releases, nor theirs behind its own)
+        if (lane == 0) {
+            int i = 0;
+            bool ok = true;
+            for (; i < nk; ++i) {
+                const int sr = i % kGemmRStages;
+                if (i >= kGemmRStages && !mbar_wait(&r_empty[sr], (uint32_t)(((i / kGemmRStages) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                const int gi = kb + i;  // global k step
                 const int j0 = 2 * gi, j1 = min(j0 + 2, nb);
                 const int r0 = s_offs[j0], rows = s_offs[j1] - r0;
                 const int g = (gi * kGemmBK) / 128;
@@ -349,8 +373,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             if (!ok) {  // let every issued copy land before the CTA can exit
                 s_misc[1] = 1;
-                for (int k = max(0, i - kGemmAStages); k < i; ++k)
-                    mbar_wait(&a_full[k % kGemmAStages], (uint32_t)((k / kGemmAStages) & 1));
                 for (int k = max(0, i - kGemmRStages); k < i; ++k)
                     mbar_wait(&r_full[k % kGemmRStages], (uint32_t)((k / kGemmRStages) & 1));
             }
