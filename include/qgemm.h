@@ -105,11 +105,14 @@ size_t qgemm_scale_bytes(int K, int N);
  * device.  Synchronises the device. Returns QGEMM_OK or QGEMM_ERR_CUDA. */
 int qgemm_device_error(int* h_code, int clear);
 
-/* Which kernel family qgemm() uses for M rows (crossovers measured on B200):
+/* Which kernel family qgemm() uses for this shape: the autotuner's recorded
+ * choice, else the built-in one (crossovers measured on B200):
  *   0 = split-K integer GEMV (M <= 4): activations rounded per (128-row group,
- *       token) to int16 with a power-of-two scale, exact int32 dot products;
- *   1 = split-K tensor-core GEMV (5 <= M <= 16): decoded fp16 codes in TMEM,
- *       tcgen05.mma against the activations;
+ *       token) to int16 with a power-of-two scale (plus a second, 2^15-finer
+ *       part for the blocks next to an outlier activation), exact int32 dot
+ *       products;
+ *   1 = split-K tensor-core GEMV (5 <= M <= 16): the exact fp16 (q - z) 2^P
+ *       codes in TMEM, tcgen05.mma against the activations;
  *   2 = tcgen05 tensor-core GEMM with dequantisation into shared memory
  *       (M > 16, and 12 <= M <= 16 when its output tiles are too few to fill
  *       the GPU and it splits k across the SMs). */

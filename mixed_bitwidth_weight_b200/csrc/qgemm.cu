@@ -29,6 +29,7 @@ struct DeviceInfo {
     bool gemv_attr[2] = {false, false};
     bool int_attr[3] = {false, false, false};
     bool gemm_attr[2] = {false, false};
+    bool quant_attr = false;
 };
 
 DeviceInfo g_devs[64];
@@ -1116,12 +1117,11 @@ int qgemm_quantize(const uint16_t* d_w, const uint8_t* d_bits, int K, int N, uin
     DeviceInfo* dev = nullptr;
     if ((st = current_device_info(&dev)) != QGEMM_OK) return st;
     const size_t smem = quant_scan_smem(K);
-    static bool attr = false;  // the limit is the same on every device
-    if (!attr) {
+    if (!dev->quant_attr) {  // a per-device setting
         if (cudaFuncSetAttribute(quant_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
             cudaSuccess)
             return QGEMM_ERR_CUDA;
-        attr = true;
+        dev->quant_attr = true;
     }
     if (smem > (size_t)227 * 1024) return QGEMM_ERR_UNSUPPORTED;
     uint8_t* w8 = static_cast<uint8_t*>(d_ws);
