@@ -27,34 +27,42 @@ QG_DEV bool block_schedule_ok(const uint8_t* bits, const int32_t* offs, int j, i
 }
 
 // ------------------------------------------------------------------ pack
-// One thread per (block, column): gathers the block's 32 codes of its column
-// and emits b words of the little-endian stream.
+// One thread per (block, 4 consecutive columns): reads the block's 32 rows of
+// its 4 codes as one 32-bit word each (128 bytes per warp per row) and emits
+// the 4 columns' little-endian streams, one 16-byte store per word row.
+// N is a multiple of 8, so a thread's 4 columns are all in range.
 __global__ void __launch_bounds__(128) pack_kernel(const uint8_t* __restrict__ codes,
                                                    const uint8_t* __restrict__ bits,
                                                    const int32_t* __restrict__ offs, int K,
                                                    int N, int64_t qw_rows,
                                                    uint32_t* __restrict__ qw) {
-    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    const int n0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
     const int j = blockIdx.y;
     const int nb = K / kBlockRows;
-    if (n >= N) return;
+    if (n0 >= N) return;
     int b, off;
     if (!block_schedule_ok(bits, offs, j, nb, qw_rows, &b, &off)) {
         set_dev_error(QGEMM_DEV_BAD_SCHEDULE);
         return;
     }
     const uint32_t mask = (1u << b) - 1u;
-    const uint8_t* src = codes + (size_t)j * kBlockRows * N + n;
-    uint32_t* dst = qw + (size_t)off * N + n;
-    uint64_t acc = 0;
+    const uint8_t* src = codes + (size_t)j * kBlockRows * N + n0;
+    uint32_t* dst = qw + (size_t)off * N + n0;
+    uint32_t rows[kBlockRows];
+#pragma unroll
+    for (int r = 0; r < kBlockRows; ++r) rows[r] = *reinterpret_cast<const uint32_t*>(src + (size_t)r * N);
+    uint64_t acc[4] = {0, 0, 0, 0};
     int nacc = 0, w = 0;
 #pragma unroll
     for (int r = 0; r < kBlockRows; ++r) {
-        acc |= (uint64_t)(src[(size_t)r * N] & mask) << nacc;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[c] |= (uint64_t)((rows[r] >> (8 * c)) & mask) << nacc;
         nacc += b;
         if (nacc >= 32) {
-            dst[(size_t)w * N] = (uint32_t)acc;
-            acc >>= 32;
+            *reinterpret_cast<uint4*>(dst + (size_t)w * N) =
+                make_uint4((uint32_t)acc[0], (uint32_t)acc[1], (uint32_t)acc[2], (uint32_t)acc[3]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[c] >>= 32;
             nacc -= 32;
             ++w;
         }

@@ -985,7 +985,7 @@ int qgemm_pack(const uint8_t* d_codes, const uint8_t* d_bits, const int32_t* d_o
     if (st != QGEMM_OK) return st;
     if ((st = check_rows(K, qw_rows)) != QGEMM_OK) return st;
     if (!aligned16(d_codes) || !aligned16(d_qw)) return QGEMM_ERR_ALIGN;
-    const dim3 grid((N + 127) / 128, K / kBlockRows);
+    const dim3 grid((N / 4 + 127) / 128, K / kBlockRows);
     pack_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(d_codes, d_bits, d_offs, K, N,
                                                                       qw_rows, d_qw);
     return launch_status();

@@ -43,6 +43,21 @@ def test_pack_bit_exact(q, K, N, kind):
     assert np.array_equal(qw.cpu().numpy().view(np.uint32), pr["qw"])
 
 
+def test_pack_ignores_bits_above_the_width(q):
+    """Codes wider than their block's width: only the low b bits are packed."""
+    import oracle
+    K, N = 1024, 1032
+    pr = P.make(K, N, kind="shuffled", seed=5)
+    rng = np.random.default_rng(6)
+    wide = rng.integers(0, 256, size=pr["codes"].shape, dtype=np.uint8)
+    widths = np.repeat(pr["bits"].astype(np.int64), 32)[:, None]
+    low = (wide & ((1 << widths) - 1)).astype(np.uint8)
+    g = P.to_gpu(pr)
+    qw = torch.full((int(pr["offs"][-1]), N), -1, dtype=torch.int32, device="cuda")
+    q.qgemm_pack(torch.as_tensor(wide).cuda(), g["bits"], g["offs"], qw)
+    assert np.array_equal(qw.cpu().numpy().view(np.uint32), oracle.pack(low, pr["bits"]))
+
+
 @pytest.mark.parametrize("K,N", SHAPES)
 @pytest.mark.parametrize("kind", KINDS)
 def test_dequant_bit_exact(q, K, N, kind):
