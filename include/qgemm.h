@@ -213,8 +213,9 @@ double qgemm_iqm(const float* h_values, int n);
  *   d_v      [nvec][D] fp16 (in for quantise, out for dequantise);
  *   d_codes  [nvec][D/32][bits] uint32;  d_scales [nvec][D/32] fp16;
  *   bits     2, 3, 4, 5, 6 or 8 (QGEMM_ERR_BITS otherwise).
- * Pointers: d_codes 4-byte aligned, the fp16 arrays 2-byte aligned.  Finite
- * inputs only.  Asynchronous on `stream`; nvec = 0 launches nothing. */
+ * Pointers: d_v 8-byte aligned (each lane moves D/32 consecutive elements in
+ * one access), d_codes 4-byte, d_scales 2-byte (QGEMM_ERR_ALIGN otherwise).
+ * Finite inputs only.  Asynchronous on `stream`; nvec = 0 launches nothing. */
 int qgemm_kv_quantize(const uint16_t* d_v, int64_t nvec, int D, int bits, uint32_t* d_codes,
                       uint16_t* d_scales, void* stream);
 int qgemm_kv_dequantize(const uint32_t* d_codes, const uint16_t* d_scales, int64_t nvec, int D, int bits,

@@ -646,8 +646,12 @@ __global__ void __launch_bounds__(kIntThreads, MP <= 2 ? 2 : 1)
                                       int_acc_shift(b) + 15 * part;
                         const int e1 = e / 2, e2 = e - e / 2;
                         const float f1 = __int_as_float((127 - e1) << 23), f2 = __int_as_float((127 - e2) << 23);
+                        // acc * (sc * 2^-e1) rounds as (acc * sc) * 2^-e1, and the
+                        // exact scaling by 2^-e2 fuses with the add: the same bits
+                        // as multiplying out and adding, in fewer instructions
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) yacc[q][ps * TP + tt] += ((float)acc[q][tt] * sc[q]) * f1 * f2;
+                        for (int q = 0; q < 4; ++q)
+                            yacc[q][ps * TP + tt] = fmaf((float)acc[q][tt] * (sc[q] * f1), f2, yacc[q][ps * TP + tt]);
                     }
                 }
             }

@@ -12,12 +12,13 @@
 //             code r at bits [r b, r b + b) of the LSB-first stream.
 // Dequantise: u' = (q - 2^(b-1)) s, v' = fp16((H_D u') / D)  (H_D H_D = D I).
 //
-// Each warp takes kKvPerWarp consecutive vectors and issues all their loads
-// before any arithmetic; lane l holds elements l + 32 r, r = 0 .. D/32 - 1, so
-// group r is register r across the warp.  The fast Walsh-Hadamard transform
-// runs in single precision in the order strides 1, 2, ..., D/2, each stage
-// replacing (a at i, b at i + stride) by (a + b, a - b): strides below 32 pair
-// lanes (shuffles), larger strides pair registers.  Every operation rounds to
+// One warp per vector; lane l holds E = D/32 consecutive elements (vector
+// loads and stores), so a group of 32 elements is 32/E consecutive lanes: its
+// largest magnitude and its packed words come from a few lane shuffles.  The
+// fast Walsh-Hadamard transform runs in single precision in the order strides
+// 1, 2, ..., D/2, each stage replacing (a at i, b at i + stride) by
+// (a + b, a - b): strides below E pair a lane's registers, larger ones pair
+// lanes.  Every operation rounds to
 // nearest even, so the codes are the same bits as any implementation of the
 // same steps.  Both kernels read and write each byte once (HBM-bound).
 #pragma once
@@ -26,127 +27,130 @@
 
 namespace qg {
 
-constexpr int kKvWarps = 8;    // warps per CTA
-constexpr int kKvPerWarp = 1;  // vectors per warp (measured: four per warp, loads first, was slower)
+constexpr int kKvWarps = 8;  // vectors per CTA (one per warp)
 
-template <int R>
-QG_DEV void fwht_warp(float (&x)[R], int lane) {
+// Fast Walsh-Hadamard transform of one vector held by a warp, E = D / 32
+// consecutive elements per lane (lane l holds elements E l .. E l + E - 1):
+// strides below E pair registers of a lane, larger strides pair lanes
+// (shuffles); the stages run in stride order 1, 2, 4, ...
+template <int E>
+QG_DEV void fwht_warp(float (&x)[E], int lane) {
 #pragma unroll
-    for (int st = 1; st < 32; st <<= 1) {
-        const bool hi = (lane & st) != 0;
+    for (int st = 1; st < E; st <<= 1)
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const float o = __shfl_xor_sync(0xffffffffu, x[r], st);
-            x[r] = hi ? __fsub_rn(o, x[r]) : __fadd_rn(x[r], o);
+        for (int i = 0; i < E; ++i)
+            if (!(i & st)) {
+                const float a = x[i], c = x[i + st];
+                x[i] = __fadd_rn(a, c);
+                x[i + st] = __fsub_rn(a, c);
+            }
+#pragma unroll
+    for (int ls = 1; ls < 32; ls <<= 1) {  // element stride E * ls
+        const bool hi = (lane & ls) != 0;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[i], ls);
+            x[i] = hi ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
         }
     }
-#pragma unroll
-    for (int sr = 1; sr < R; sr <<= 1)
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-            if (!(r & sr)) {
-                const float a = x[r], c = x[r + sr];
-                x[r] = __fadd_rn(a, c);
-                x[r + sr] = __fsub_rn(a, c);
-            }
 }
 
-template <int R>
+// Groups of 32 elements are 32 / E consecutive lanes; lane-in-group g = lane % (32 / E).
+template <int E>
 __global__ void __launch_bounds__(32 * kKvWarps) kv_quant_kernel(const __half* __restrict__ v, int64_t nvec, int b,
                                                                 uint32_t* __restrict__ codes,
                                                                 __half* __restrict__ scales) {
-    constexpr int D = 32 * R;
+    constexpr int D = 32 * E, G = 32 / E;  // lanes per group
     const int lane = threadIdx.x & 31;
-    const int64_t t0 = ((int64_t)blockIdx.x * kKvWarps + (threadIdx.x >> 5)) * kKvPerWarp;
-    if (t0 >= nvec) return;  // whole warps only
-    const int nv = (nvec - t0 < kKvPerWarp) ? (int)(nvec - t0) : kKvPerWarp;
-    // every load of the warp's vectors first, then the arithmetic
-    float x[kKvPerWarp][R];
+    const int64_t t = (int64_t)blockIdx.x * kKvWarps + (threadIdx.x >> 5);
+    if (t >= nvec) return;  // whole warps only
+    float x[E];
+    const __half* src = v + t * D + E * lane;
+    if constexpr (E == 1) {
+        x[0] = __half2float(src[0]);
+    } else if constexpr (E == 2) {
+        const __half2 h = *reinterpret_cast<const __half2*>(src);
+        x[0] = __low2float(h);
+        x[1] = __high2float(h);
+    } else {
 #pragma unroll
-    for (int j = 0; j < kKvPerWarp; ++j)
-#pragma unroll
-        for (int r = 0; r < R; ++r) x[j][r] = (j < nv) ? __half2float(v[(t0 + j) * D + 32 * r + lane]) : 0.f;
-    const int z = 1 << (b - 1);
-#pragma unroll
-    for (int j = 0; j < kKvPerWarp; ++j) {
-        if (j >= nv) break;  // uniform over the warp
-        const int64_t t = t0 + j;
-        fwht_warp<R>(x[j], lane);
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            float amax = fabsf(x[j][r]);
-#pragma unroll
-            for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            const __half sh = __float2half_rn(__fdiv_rn(amax, (float)(z - 1)));
-            const float s = __half2float(sh);
-            int q = z;
-            if (s != 0.f) {
-                float tq = rintf(__fmul_rn(x[j][r], __fdiv_rn(1.f, s)));
-                if (tq != tq) tq = 0.f;  // not a number: the zero point
-                tq = fminf(fmaxf(tq, (float)(-z)), (float)(z - 1));
-                q = (int)tq + z;
-            }
-            uint32_t* w = codes + (t * R + r) * b;
-            uint32_t mine = 0;  // lane k keeps word k
-            for (int k = 0; k < b; ++k) {
-                const int d = lane * b - 32 * k;  // the code's first bit, relative to word k
-                uint32_t part = 0;
-                if (d >= 0 && d < 32) part = (uint32_t)q << d;
-                else if (d < 0 && d + b > 0) part = (uint32_t)q >> (-d);
-                part = __reduce_or_sync(0xffffffffu, part);
-                if (lane == k) mine = part;
-            }
-            if (lane < b) w[lane] = mine;
-            if (lane == 0) scales[t * R + r] = sh;
+        for (int i = 0; i < E; i += 4) {
+            const uint2 u = *reinterpret_cast<const uint2*>(src + i);
+            x[i] = __low2float(*reinterpret_cast<const __half2*>(&u.x));
+            x[i + 1] = __high2float(*reinterpret_cast<const __half2*>(&u.x));
+            x[i + 2] = __low2float(*reinterpret_cast<const __half2*>(&u.y));
+            x[i + 3] = __high2float(*reinterpret_cast<const __half2*>(&u.y));
         }
     }
+    fwht_warp<E>(x, lane);
+    const int z = 1 << (b - 1);
+    const int grp = lane / G, gl = lane % G;  // group of this lane, lane within it
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const __half sh = __float2half_rn(__fdiv_rn(amax, (float)(z - 1)));
+    const float s = __half2float(sh);
+    const float inv = (s == 0.f) ? 0.f : __fdiv_rn(1.f, s);
+    // this lane's E codes: bits [E gl b, E gl b + E b) of its group's stream
+    uint64_t chunk = 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        int q = z;
+        if (s != 0.f) {
+            float tq = rintf(__fmul_rn(x[i], inv));
+            if (tq != tq) tq = 0.f;  // not a number: the zero point
+            tq = fminf(fmaxf(tq, (float)(-z)), (float)(z - 1));
+            q = (int)tq + z;
+        }
+        chunk |= (uint64_t)q << (i * b);
+    }
+    const int pos = E * gl * b;  // first stream bit of the chunk
+    uint32_t* w = codes + (t * E + grp) * b;
+    for (int k = 0; k < b; ++k) {
+        const int d = pos - 32 * k;  // the chunk's first bit, relative to word k
+        uint32_t part = 0;
+        if (d >= 0 && d < 32) part = (uint32_t)(chunk << d);
+        else if (d < 0 && d + E * b > 0) part = (uint32_t)(chunk >> (-d));
+#pragma unroll
+        for (int o = 1; o < G; o <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, o);
+        if (gl == k % G) w[k] = part;
+    }
+    if (gl == 0) scales[t * E + grp] = sh;
 }
 
-template <int R>
+template <int E>
 __global__ void __launch_bounds__(32 * kKvWarps) kv_dequant_kernel(const uint32_t* __restrict__ codes,
                                                                   const __half* __restrict__ scales, int64_t nvec,
                                                                   int b, __half* __restrict__ v) {
-    constexpr int D = 32 * R;
+    constexpr int D = 32 * E, G = 32 / E;
     const int lane = threadIdx.x & 31;
-    const int64_t t0 = ((int64_t)blockIdx.x * kKvWarps + (threadIdx.x >> 5)) * kKvPerWarp;
-    if (t0 >= nvec) return;
-    const int nv = (nvec - t0 < kKvPerWarp) ? (int)(nvec - t0) : kKvPerWarp;
+    const int64_t t = (int64_t)blockIdx.x * kKvWarps + (threadIdx.x >> 5);
+    if (t >= nvec) return;
     const int z = 1 << (b - 1);
-    const uint32_t mask = (1u << b) - 1u;
-    const int p = lane * b, wi = p >> 5, o = p & 31;
-    const bool two = o + b > 32;  // the code straddles two words
-    // every load of the warp's vectors first (the words holding this lane's
-    // codes and the group scales), then the arithmetic
-    uint32_t lo[kKvPerWarp][R], hi[kKvPerWarp][R];
-    float sc[kKvPerWarp][R];
+    const int grp = lane / G, gl = lane % G;
+    const uint32_t* w = codes + (t * E + grp) * b;
+    const int pos = E * gl * b, wi = pos >> 5, o = pos & 31;
+    // the chunk spans at most three words (E b <= 64 bits)
+    const uint64_t lo = w[wi] | ((wi + 1 < b) ? (uint64_t)w[wi + 1] << 32 : 0ull);
+    uint64_t chunk = lo >> o;
+    if (o > 0 && wi + 2 < b) chunk |= (uint64_t)w[wi + 2] << (64 - o);
+    const float s = __half2float(scales[t * E + grp]);
+    const uint64_t mask = (1ull << b) - 1ull;
+    float x[E];
 #pragma unroll
-    for (int j = 0; j < kKvPerWarp; ++j)
+    for (int i = 0; i < E; ++i) x[i] = __fmul_rn((float)((int)((chunk >> (i * b)) & mask) - z), s);  // exact
+    fwht_warp<E>(x, lane);
+    __half* dst = v + t * D + E * lane;
+    const float inv_d = 1.f / (float)D;  // a power of two: exact
+    if constexpr (E == 1) {
+        dst[0] = __float2half_rn(__fmul_rn(x[0], inv_d));
+    } else {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            lo[j][r] = hi[j][r] = 0u;
-            sc[j][r] = 0.f;
-            if (j < nv) {
-                const uint32_t* w = codes + ((t0 + j) * R + r) * b;
-                lo[j][r] = w[wi];
-                if (two) hi[j][r] = w[wi + 1];
-                sc[j][r] = __half2float(scales[(t0 + j) * R + r]);
-            }
-        }
-#pragma unroll
-    for (int j = 0; j < kKvPerWarp; ++j) {
-        if (j >= nv) break;  // uniform over the warp
-        float x[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            uint32_t q = lo[j][r] >> o;
-            if (two) q |= hi[j][r] << (32 - o);
-            q &= mask;
-            x[r] = __fmul_rn((float)((int)q - z), sc[j][r]);  // exact
-        }
-        fwht_warp<R>(x, lane);
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-            v[(t0 + j) * D + 32 * r + lane] = __float2half_rn(__fmul_rn(x[r], 1.f / (float)D));
+        for (int i = 0; i < E; i += 2)
+            *reinterpret_cast<__half2*>(dst + i) =
+                __floats2half2_rn(__fmul_rn(x[i], inv_d), __fmul_rn(x[i + 1], inv_d));
     }
 }
 

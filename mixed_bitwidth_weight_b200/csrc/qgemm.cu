@@ -1153,10 +1153,9 @@ int qgemm_kv_quantize(const uint16_t* d_v, int64_t nvec, int D, int bits, uint32
     if (nvec < 0 || nvec > ((int64_t)1 << 36) || (D != 32 && D != 64 && D != 128 && D != 256))
         return QGEMM_ERR_SHAPE;
     if (!(bits == 2 || bits == 3 || bits == 4 || bits == 5 || bits == 6 || bits == 8)) return QGEMM_ERR_BITS;
-    if (((uintptr_t)d_v & 1) || ((uintptr_t)d_codes & 3) || ((uintptr_t)d_scales & 1)) return QGEMM_ERR_ALIGN;
+    if (((uintptr_t)d_v & 7) || ((uintptr_t)d_codes & 3) || ((uintptr_t)d_scales & 1)) return QGEMM_ERR_ALIGN;
     if (nvec == 0) return QGEMM_OK;
-    const int64_t per_cta = (int64_t)kKvWarps * kKvPerWarp;
-    const dim3 grid((unsigned)((nvec + per_cta - 1) / per_cta)), block(32 * kKvWarps);
+    const dim3 grid((unsigned)((nvec + kKvWarps - 1) / kKvWarps)), block(32 * kKvWarps);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const __half* v = reinterpret_cast<const __half*>(d_v);
     __half* sc = reinterpret_cast<__half*>(d_scales);
@@ -1175,10 +1174,9 @@ int qgemm_kv_dequantize(const uint32_t* d_codes, const uint16_t* d_scales, int64
     if (nvec < 0 || nvec > ((int64_t)1 << 36) || (D != 32 && D != 64 && D != 128 && D != 256))
         return QGEMM_ERR_SHAPE;
     if (!(bits == 2 || bits == 3 || bits == 4 || bits == 5 || bits == 6 || bits == 8)) return QGEMM_ERR_BITS;
-    if (((uintptr_t)d_v & 1) || ((uintptr_t)d_codes & 3) || ((uintptr_t)d_scales & 1)) return QGEMM_ERR_ALIGN;
+    if (((uintptr_t)d_v & 7) || ((uintptr_t)d_codes & 3) || ((uintptr_t)d_scales & 1)) return QGEMM_ERR_ALIGN;
     if (nvec == 0) return QGEMM_OK;
-    const int64_t per_cta = (int64_t)kKvWarps * kKvPerWarp;
-    const dim3 grid((unsigned)((nvec + per_cta - 1) / per_cta)), block(32 * kKvWarps);
+    const dim3 grid((unsigned)((nvec + kKvWarps - 1) / kKvWarps)), block(32 * kKvWarps);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     __half* v = reinterpret_cast<__half*>(d_v);
     const __half* sc = reinterpret_cast<const __half*>(d_scales);

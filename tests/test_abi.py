@@ -220,6 +220,8 @@ def test_kv_cache_entry_points_check_arguments_on_the_host():
     assert lib.qgemm_kv_quantize(dummy, -1, 128, 4, dummy, dummy, None) == -2     # negative count
     assert lib.qgemm_kv_quantize(dummy, 1, 128, 7, dummy, dummy, None) == -3      # width
     assert lib.qgemm_kv_quantize(P(17), 1, 128, 4, dummy, dummy, None) == -4      # alignment
+    assert lib.qgemm_kv_quantize(P(4100), 1, 128, 4, dummy, dummy, None) == -4    # fp16 vectors: 8 bytes
+    assert lib.qgemm_kv_dequantize(dummy, dummy, 1, 128, 4, P(4100), None) == -4
     assert lib.qgemm_kv_dequantize(dummy, dummy, 1, 512, 4, dummy, None) == -2
     assert lib.qgemm_kv_dequantize(dummy, dummy, 1, 128, 1, dummy, None) == -3
     assert lib.qgemm_kv_quantize(dummy, 0, 128, 4, dummy, dummy, None) == 0       # nothing to do
