@@ -83,18 +83,20 @@ struct XpermParams {
     int M, K, x_bf16;
 };
 
+// Codes paired into one fp16x2 word by the dequantiser: pair i of a block
+// holds codes r = 2m (i / m) + i % m (low half) and r + m (high half), so
+// that one 32-bit window of the block's bit stream holds both, r at window
+// bit kl and r + m at bit 16 + kh (pair_kl / pair_kh below): m = 8, 4, 2 for
+// b = 2, 4, 8 (the codes 16 bits apart), m = 4 for b = 3 and 5, 2 for b = 6.
+QG_DEV constexpr int pair_m(int b) { return b == 2 ? 8 : (b == 6 || b == 8) ? 2 : 4; }
+QG_DEV constexpr int pair_kl(int b) { return (b == 3 || b == 6) ? 4 : 0; }
+QG_DEV constexpr int pair_kh(int b) { return b == 5 ? 4 : 0; }
+
 // Order of the k positions of one 32-row block inside the B tile (and so in
-// x_p): the dequantiser extracts two codes per 32-bit word into the two fp16
-// halves with one shift and one mask, so position pair i holds codes that sit
-// 16 bits apart.  b = 2: pair (8w+s) = codes (16w+s, 16w+s+8); b = 4: pair
-// (4w+s) = codes (8w+s, 8w+s+4); b = 8: pair (2w+s) = codes (4w+s, 4w+s+2);
-// 3, 5, 6: natural order.
+// x_p): position 2i + h holds code r + h m of pair i.
 QG_DEV int gemm_code_of_k(int b, int k) {
-    const int i = k >> 1, h = k & 1;
-    if (b == 2) return 16 * (i >> 3) + (i & 7) + 8 * h;
-    if (b == 4) return 8 * (i >> 2) + (i & 3) + 4 * h;
-    if (b == 8) return 4 * (i >> 1) + (i & 1) + 2 * h;
-    return k;
+    const int i = k >> 1, h = k & 1, m = pair_m(b);
+    return 2 * m * (i / m) + i % m + m * h;
 }
 
 // x_p[m][k] = fp16(x[m][perm[k']] * 2^-shift[m]), k' = the code the B tile
@@ -179,37 +181,50 @@ QG_DEV uint32_t h2mul(uint32_t a, uint32_t b) {
 }
 
 // The 32 codes of one block for this thread's column, dequantised to fp16
-// pairs in the B tile's order (gemm_code_of_k).  Two codes at bits p and
-// p + 16 of a word become (1024 + q) in each half with one mask and an OR of
-// 0x6400 (the fp16 of 1024); subtracting 1024 + z is exact and the multiply
-// by the fp16 scale is the one rounding: bit-exact with qgemm_dequant.
+// pairs in the B tile's order (gemm_code_of_k).  A code at bit k of a half
+// (k + b <= 10) becomes 2^(10-k) + q with one mask and an OR of the fp16 of
+// 2^(10-k) (0x6400 for 1024 at k = 0, 0x5400 for 64 at k = 4): its mantissa
+// step there is 1.  So each pair costs one shift (or funnel shift) of the
+// block's words, one mask-and-OR, an exact subtraction of the fp16 of
+// 2^(10-k) + z and the multiply by the fp16 scale, the one rounding:
+// bit-exact with qgemm_dequant.
 // w0 = word row 0 of the block at this column, word rows 1 KB apart.
 template <int B>
 QG_DEV void dequant_block32(const uint8_t* w0, uint32_t s2, uint32_t (&out)[16]) {
     constexpr uint32_t mask = (1u << B) - 1u;
-    const uint32_t zoff = 0x64006400u + (((uint32_t)1 << (B - 1)) * 0x00010001u);  // 1024 + z in both halves
     uint32_t w[B];
 #pragma unroll
     for (int i = 0; i < B; ++i) w[i] = *reinterpret_cast<const uint32_t*>(w0 + i * 1024);
     if constexpr (B == 2 || B == 4 || B == 8) {
         constexpr int per = 16 / B;  // pairs per word
+        const uint32_t zoff = 0x64006400u + (((uint32_t)1 << (B - 1)) * 0x00010001u);  // 1024 + z in both halves
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int wi = i / per, sft = (i % per) * B;
             const uint32_t h = lop3_and_or(w[wi] >> sft, mask * 0x00010001u, 0x64006400u);
             out[i] = h2mul(h2sub(h, zoff), s2);
         }
-    } else {  // 3, 5, 6: codes 2i and 2i+1 in natural order
+    } else {  // 3, 5, 6: window at stream bit b r - kl (below 0: shifted in zeros)
+        constexpr int m = pair_m(B), kl = pair_kl(B), kh = pair_kh(B);
+        constexpr uint32_t mlo = kl ? 0x5400u : 0x6400u, mhi = kh ? 0x5400u : 0x6400u;
+        constexpr uint32_t pmask = (mask << kl) | (mask << (16 + kh));
+        constexpr uint32_t magic = mlo | (mhi << 16);
+        constexpr uint32_t z = 1u << (B - 1);
+        const uint32_t zpair = (mlo + (z << kl)) | ((mhi + (z << kh)) << 16);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            uint32_t q[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int bit = (2 * i + u) * B, wi = bit >> 5, sh = bit & 31;
-                if (sh + B <= 32) q[u] = (w[wi] >> sh) & mask;
-                else q[u] = __funnelshift_r(w[wi], w[wi + 1 < B ? wi + 1 : wi], sh) & mask;
+            const int r = 2 * m * (i / m) + i % m;
+            const int base = B * r - kl, end = B * (r + m) + B;  // window start, last bit used + 1
+            uint32_t v;
+            if (base < 0) {
+                v = w[0] << (-base);
+            } else {
+                const int wi = base >> 5, sh = base & 31;
+                if (sh == 0) v = w[wi];
+                else if (end <= 32 * (wi + 1)) v = w[wi] >> sh;
+                else v = __funnelshift_r(w[wi], w[wi + 1 < B ? wi + 1 : wi], sh);
             }
-            out[i] = h2mul(h2sub((q[0] | (q[1] << 16)) | 0x64006400u, zoff), s2);
+            out[i] = h2mul(h2sub(lop3_and_or(v, pmask, magic), zpair), s2);
         }
     }
 }

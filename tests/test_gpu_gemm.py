@@ -143,3 +143,33 @@ def test_gemm_prefill_layer_sampled_columns(q):
     yg = y[:, torch.as_tensor(cols, device="cuda")]
     # rms over the sampled outputs stands in for the whole output's rms
     P.check_close(yg, yr)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 48, 64])
+@pytest.mark.parametrize("knob", [1, 4])
+def test_gemm_few_rows_forced(q, M, knob):
+    """The GEMM at few rows of x (the MMA operands swapped, N = M rounded up
+    to 16), chosen through a recorded tuning entry: whole tiles (knob 1) and
+    k split four ways (knob 4); fp16 and bf16 input; one-hot rows exact."""
+    K, N = 1024, 776
+    try:
+        q.qgemm_tune_record(M, K, N, 2, knob)
+        for x_dtype in (torch.float16, torch.bfloat16):
+            pr = P.make(K, N, M=M, kind="shuffled", seed=M + knob, x_dtype=x_dtype)
+            g = P.to_gpu(pr)
+            y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+            q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, q.workspace(M, K, N))
+            torch.cuda.synchronize()
+            P.check_close(y, P.ref_y(pr))
+        rng = np.random.default_rng(M)
+        js = rng.integers(0, K, size=M)
+        x = torch.zeros(M, K, dtype=torch.float16)
+        x[np.arange(M), js] = 1.0
+        pr["x"] = x
+        g = P.to_gpu(pr)
+        q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, q.workspace(M, K, N))
+        w16 = oracle.dequant_f16(pr["qw"], pr["scales"].numpy(), pr["bits"], K)
+        inv = np.argsort(pr["perm"])
+        assert np.array_equal(y.cpu().numpy().view(np.uint16), w16[inv[js]])
+    finally:
+        q.qgemm_tune_clear()
