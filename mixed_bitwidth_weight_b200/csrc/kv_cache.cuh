@@ -13,8 +13,11 @@
 // Dequantise: u' = (q - 2^(b-1)) s, v' = fp16((H_D u') / D)  (H_D H_D = D I).
 //
 // One warp per vector; lane l holds E = D/32 consecutive elements (vector
-// loads and stores), so a group of 32 elements is 32/E consecutive lanes: its
-// largest magnitude and its packed words come from a few lane shuffles.  The
+// loads and stores), so a group of 32 elements is 32/E consecutive lanes and
+// its largest magnitude takes log2(32/E) shuffles.  The groups' code streams
+// follow one another, so lane l's E codes are bits [E b l, E b (l + 1)) of the
+// vector's stream, and lane j assembles word j from the two to four lanes
+// whose bits it holds, one coalesced store per lane.  The
 // fast Walsh-Hadamard transform runs in single precision in the order strides
 // 1, 2, ..., D/2, each stage replacing (a at i, b at i + stride) by
 // (a + b, a - b): strides below E pair a lane's registers, larger ones pair
@@ -56,11 +59,13 @@ QG_DEV void fwht_warp(float (&x)[E], int lane) {
 }
 
 // Groups of 32 elements are 32 / E consecutive lanes; lane-in-group g = lane % (32 / E).
-template <int E>
-__global__ void __launch_bounds__(32 * kKvWarps) kv_quant_kernel(const __half* __restrict__ v, int64_t nvec, int b,
+// b = B bits per code.
+template <int E, int B>
+__global__ void __launch_bounds__(32 * kKvWarps) kv_quant_kernel(const __half* __restrict__ v, int64_t nvec,
                                                                 uint32_t* __restrict__ codes,
                                                                 __half* __restrict__ scales) {
     constexpr int D = 32 * E, G = 32 / E;  // lanes per group
+    constexpr int b = B;
     const int lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * kKvWarps + (threadIdx.x >> 5);
     if (t >= nvec) return;  // whole warps only
@@ -83,7 +88,7 @@ __global__ void __launch_bounds__(32 * kKvWarps) kv_quant_kernel(const __half* _
         }
     }
     fwht_warp<E>(x, lane);
-    const int z = 1 << (b - 1);
+    constexpr int z = 1 << (b - 1);
     const int grp = lane / G, gl = lane % G;  // group of this lane, lane within it
     float amax = 0.f;
 #pragma unroll
@@ -92,8 +97,9 @@ __global__ void __launch_bounds__(32 * kKvWarps) kv_quant_kernel(const __half* _
     for (int o = 1; o < G; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const __half sh = __float2half_rn(__fdiv_rn(amax, (float)(z - 1)));
     const float s = __half2float(sh);
-    const float inv = (s == 0.f) ? 0.f : __fdiv_rn(1.f, s);
-    // this lane's E codes: bits [E gl b, E gl b + E b) of its group's stream
+    const float inv = (s == 0.f) ? 0.f : __frcp_rn(s);  // the correctly rounded 1 / s
+    // this lane's E codes: bits [c l, c l + c) of the vector's stream, c = E b
+    // (group g's b words follow group g - 1's, so the groups' streams join)
     uint64_t chunk = 0;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
@@ -106,16 +112,28 @@ __global__ void __launch_bounds__(32 * kKvWarps) kv_quant_kernel(const __half* _
         }
         chunk |= (uint64_t)q << (i * b);
     }
-    const int pos = E * gl * b;  // first stream bit of the chunk
-    uint32_t* w = codes + (t * E + grp) * b;
-    for (int k = 0; k < b; ++k) {
-        const int d = pos - 32 * k;  // the chunk's first bit, relative to word k
-        uint32_t part = 0;
-        if (d >= 0 && d < 32) part = (uint32_t)(chunk << d);
-        else if (d < 0 && d + E * b > 0) part = (uint32_t)(chunk >> (-d));
+    // word j of the c words: the chunks of lanes floor(32 j / c) ..
+    // floor((32 j + 31) / c), at most floor(31 / c) + 2 of them; lane j
+    // gathers word j (and j + 32 when c > 32)
+    constexpr int c = E * b;
+    constexpr int nsrc = 31 / c + 2;
+    const uint32_t clo = (uint32_t)chunk, chi = (uint32_t)(chunk >> 32);
+    uint32_t* wv = codes + t * c;
 #pragma unroll
-        for (int o = 1; o < G; o <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, o);
-        if (gl == k % G) w[k] = part;
+    for (int pass = 0; pass < (E == 8 ? 2 : 1); ++pass) {
+        const int j = lane + 32 * pass;
+        const int l0 = (32 * j) / c, l1 = (32 * j + 31) / c;
+        uint32_t word = 0;
+#pragma unroll
+        for (int r = 0; r < nsrc; ++r) {
+            const int l = min(l0 + r, 31);
+            const uint32_t vlo = __shfl_sync(0xffffffffu, clo, l);
+            const uint32_t vhi = (E * 8 > 32) ? __shfl_sync(0xffffffffu, chi, l) : 0u;
+            const uint64_t v = ((uint64_t)vhi << 32) | vlo;
+            const int d = c * l - 32 * j;  // the chunk's first bit relative to the word
+            if (l0 + r <= l1) word |= (d >= 0) ? (uint32_t)(v << d) : (uint32_t)(v >> (-d));
+        }
+        if (j < c) wv[j] = word;
     }
     if (gl == 0) scales[t * E + grp] = sh;
 }

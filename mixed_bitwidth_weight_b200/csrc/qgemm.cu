@@ -844,6 +844,20 @@ int autotune_shape(const void* x, int x_dtype, const int32_t* perm, const uint32
     return rows;
 }
 
+// The KV quantiser instantiated for the code width.
+template <int E>
+void launch_kv_quant(dim3 grid, dim3 block, cudaStream_t s, const __half* v, int64_t nvec, int bits,
+                     uint32_t* codes, __half* sc) {
+    switch (bits) {
+        case 2: kv_quant_kernel<E, 2><<<grid, block, 0, s>>>(v, nvec, codes, sc); break;
+        case 3: kv_quant_kernel<E, 3><<<grid, block, 0, s>>>(v, nvec, codes, sc); break;
+        case 4: kv_quant_kernel<E, 4><<<grid, block, 0, s>>>(v, nvec, codes, sc); break;
+        case 5: kv_quant_kernel<E, 5><<<grid, block, 0, s>>>(v, nvec, codes, sc); break;
+        case 6: kv_quant_kernel<E, 6><<<grid, block, 0, s>>>(v, nvec, codes, sc); break;
+        default: kv_quant_kernel<E, 8><<<grid, block, 0, s>>>(v, nvec, codes, sc); break;
+    }
+}
+
 }  // namespace
 
 // =========================================================== C ABI
@@ -1160,10 +1174,10 @@ int qgemm_kv_quantize(const uint16_t* d_v, int64_t nvec, int D, int bits, uint32
     const __half* v = reinterpret_cast<const __half*>(d_v);
     __half* sc = reinterpret_cast<__half*>(d_scales);
     switch (D / 32) {
-        case 1: kv_quant_kernel<1><<<grid, block, 0, s>>>(v, nvec, bits, d_codes, sc); break;
-        case 2: kv_quant_kernel<2><<<grid, block, 0, s>>>(v, nvec, bits, d_codes, sc); break;
-        case 4: kv_quant_kernel<4><<<grid, block, 0, s>>>(v, nvec, bits, d_codes, sc); break;
-        default: kv_quant_kernel<8><<<grid, block, 0, s>>>(v, nvec, bits, d_codes, sc); break;
+        case 1: launch_kv_quant<1>(grid, block, s, v, nvec, bits, d_codes, sc); break;
+        case 2: launch_kv_quant<2>(grid, block, s, v, nvec, bits, d_codes, sc); break;
+        case 4: launch_kv_quant<4>(grid, block, s, v, nvec, bits, d_codes, sc); break;
+        default: launch_kv_quant<8>(grid, block, s, v, nvec, bits, d_codes, sc); break;
     }
     return launch_status();
 }
