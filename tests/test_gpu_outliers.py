@@ -76,3 +76,40 @@ def test_outlier_over_live_row(q, M):
     y = torch.empty((M, N), dtype=torch.float16, device="cuda")
     q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, q.workspace(M, K, N))
     P.check_close(y, P.ref_y(pr))
+
+
+def bf16_outlier_problem(K, N, M, mag, seed):
+    """bf16 activations with one outlier of magnitude mag per chosen group,
+    each over a zero-point weight row (as outlier_problem), so that the rest
+    of each row spans a range of mag to 1."""
+    pr, rows = outlier_problem(K, N, M, 1.0, seed)
+    x = P.make(K, N, M=M, kind="shuffled", seed=seed, x_dtype=torch.bfloat16)["x"].clone()
+    for k in rows:
+        x[:, int(pr["perm"][k])] = mag
+    pr["x"] = x
+    return pr, rows
+
+
+# The integer GEMV (M <= 4) encodes a group as int16 on the grid of its
+# largest magnitude plus a second int16 part on a grid 2^15 times finer, so a
+# value 2^24 below the group's maximum keeps about 5 bits (measured: 3.6e-2 *
+# rms at M = 1); the fp16 paths scale whole rows, exactly for every value
+# within 2^24 of the row maximum.
+BF16_RANGES = [(M, 2.0 ** 20) for M in (1, 4, 8, 13, 32, 96)] + [(M, 2.0 ** 24) for M in (8, 13, 32, 96)]
+
+
+@pytest.mark.parametrize("M,mag", BF16_RANGES)
+def test_bf16_outlier_over_zero_row(q, M, mag):
+    """bf16 input is brought to fp16 (or to integers) with a power-of-two
+    scale set by the largest magnitude of its row or group: with the rest of
+    the row 2^20 below that maximum every decode path (the integer GEMV, the
+    tensor-core GEMV and the GEMM) keeps y within the usual tolerance, and the
+    two fp16 paths still at 2^24."""
+    K, N = 4096, 520
+    pr, rows = bf16_outlier_problem(K, N, M, mag, seed=M + int(np.log2(mag)))
+    w16 = oracle.dequant_f16(pr["qw"], pr["scales"].numpy(), pr["bits"], K)
+    assert not np.any(w16[rows].view(np.uint16) & 0x7FFF), "outlier rows must dequantise to zero"
+    g = P.to_gpu(pr)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    q.qgemm(g["x"], g["perm"], g["qw"], g["scales"], g["bits"], g["offs"], y, q.workspace(M, K, N))
+    P.check_close(y, P.ref_y(pr))
